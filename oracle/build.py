@@ -1,0 +1,30 @@
+"""Compile the CPU oracle (test infrastructure) into oracle/librcoracle.so.
+
+The oracle is plain single-threaded C.  It is built with contraction and
+fast-math off, so each C `float` operation is one IEEE binary32 operation.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "rc_oracle.c")
+LIB = os.path.join(HERE, "librcoracle.so")
+
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+          "-fno-fast-math", "-fexcess-precision=standard", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Build the shared library if missing or older than its source."""
+    if (not force and os.path.exists(LIB)
+            and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
+        return LIB
+    cmd = ["gcc", *CFLAGS, "-o", LIB + ".tmp", SRC]
+    subprocess.run(cmd, check=True)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))

@@ -1,0 +1,128 @@
+"""Seeded synthetic rank buffers -- shared by the tests, the bench and smoke().
+
+This module draws random numbers and lays them out per rank.  It holds none of
+the collectives' arithmetic: no reduction, no rounding rule, no ordering.  Both
+the CPU oracle and the CUDA library consume what it returns.
+
+Each generator returns a list of ``p`` contiguous host numpy arrays, one per
+simulated rank, drawn in rank order 0..p-1 from ONE ``torch.Generator`` seeded
+with ``seed``.  Storage types: float32 ("f32"), uint16 bf16 bit patterns
+("bf16", the fp32 draw narrowed by torch's round-to-nearest-even ``.to``),
+int32 ("i32").
+
+Workloads (sizes and value distributions as the collectives' pages and their
+reproduction recipe state them):
+  * worked example: x_r = [0,1,2,3] + r, p = 4;
+  * uniform[lo, hi), normal N(0, sigma) (sigma is a standard deviation),
+    integers uniform[lo, hi);
+  * the transformer-layer parameter count 4*4096*4096 + 3*4096*11008 of a
+    Llama-2-7B decoder layer (Q, K, V, O projections and gate, up, down).
+"""
+from __future__ import annotations
+
+from typing import List
+
+import numpy as np
+import torch
+
+# Llama-2-7B decoder layer: W_Q, W_K, W_V, W_O are 4096x4096; W_gate, W_up are
+# 4096x11008 and W_down is 11008x4096.
+LLAMA2_7B_LAYER_ELEMS = 4 * 4096 * 4096 + 3 * 4096 * 11008  # 202,375,168
+
+NP = {"f32": np.float32, "bf16": np.uint16, "i32": np.int32}
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def _store(t: torch.Tensor, dt: str) -> np.ndarray:
+    if dt == "f32":
+        return t.to(torch.float32).contiguous().numpy()
+    if dt == "bf16":
+        return t.to(torch.float32).to(torch.bfloat16).view(torch.int16).contiguous().numpy().view(np.uint16)
+    if dt == "i32":
+        return t.to(torch.int32).contiguous().numpy()
+    raise ValueError(dt)
+
+
+def worked_example(p: int = 4, n: int = 4, dt: str = "f32") -> List[np.ndarray]:
+    """x_r[i] = i + r (the pages' four-rank example for n = 4)."""
+    return [_store(torch.arange(n, dtype=torch.float64) + r, dt) if dt != "i32"
+            else (np.arange(n, dtype=np.int64) + r).astype(np.int32) for r in range(p)]
+
+
+def uniform(p: int, n: int, seed: int, dt: str = "f32", lo: float = -1.0, hi: float = 1.0) -> List[np.ndarray]:
+    g = _gen(seed)
+    out = []
+    for _ in range(p):
+        t = torch.rand(n, generator=g, dtype=torch.float32) * (hi - lo) + lo
+        out.append(_store(t, dt))
+    return out
+
+
+def normal(p: int, n: int, seed: int, sigma: float = 1.0, dt: str = "f32") -> List[np.ndarray]:
+    g = _gen(seed)
+    out = []
+    for _ in range(p):
+        t = torch.randn(n, generator=g, dtype=torch.float32) * sigma
+        out.append(_store(t, dt))
+    return out
+
+
+def int_uniform(p: int, n: int, seed: int, lo: int = -(1 << 20), hi: int = 1 << 20) -> List[np.ndarray]:
+    g = _gen(seed)
+    return [torch.randint(lo, hi, (n,), generator=g, dtype=torch.int32).numpy() for _ in range(p)]
+
+
+def sweep_data(p: int, n: int, seed: int, dt: str) -> List[np.ndarray]:
+    """The sweep's value distributions: floats uniform[-1,1), ints uniform[-2^20, 2^20)."""
+    if dt == "i32":
+        return int_uniform(p, n, seed)
+    return uniform(p, n, seed, dt)
+
+
+def special_values(p: int, n: int, seed: int, dt: str = "f32") -> List[np.ndarray]:
+    """Values that stress ordering and rounding: signed zeros, large/small
+    magnitudes that cancel, exact powers of two, bf16 rounding ties."""
+    rng = np.random.default_rng(seed)
+    if dt == "i32":
+        pool = np.array([0, 1, -1, 2**31 - 1, -2**31, 2**30, -2**30, 12345, -7], dtype=np.int64)
+        return [pool[rng.integers(0, pool.size, n)].astype(np.int32) for _ in range(p)]
+    pool = np.array([0.0, -0.0, 1.0, -1.0, 2.0**24, -2.0**24, 2.0**-24, 3.0, 1e-3, -1e-3,
+                     1.0 + 2.0**-8, 1.0 + 3 * 2.0**-9, 65504.0, -0.5, 2.0**-126, 7.25e9],
+                    dtype=np.float32)
+    out = []
+    for _ in range(p):
+        v = pool[rng.integers(0, pool.size, n)]
+        if dt == "f32":
+            out.append(v.astype(np.float32))
+        else:
+            out.append(_store(torch.from_numpy(v.astype(np.float32)), "bf16"))
+    return out
+
+
+def config(name: str):
+    """The five named workloads: a dict with everything needed to draw them."""
+    cfgs = {
+        "worked_example": dict(p=4, n=4, dt="f32", gen="worked"),
+        "cfg1": dict(p=4, n=65536, dt="f32", gen="uniform", seed=0),
+        "cfg2_ring": dict(p=8, n=2097152, dt="f32", gen="normal", seed=1, sigma=1e-2),
+        "cfg3_hier": dict(p=8, n=4194304, dt="bf16", gen="normal", seed=2, sigma=1.0, group=4),
+        "cfg4_params": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS // 8, dt="bf16", gen="uniform", seed=3),
+        "cfg4_grads": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS, dt="f32", gen="normal", seed=4, sigma=1e-3),
+    }
+    return cfgs[name]
+
+
+def draw(cfg: dict) -> List[np.ndarray]:
+    g = cfg["gen"]
+    if g == "worked":
+        return worked_example(cfg["p"], cfg["n"], cfg["dt"])
+    if g == "uniform":
+        return uniform(cfg["p"], cfg["n"], cfg["seed"], cfg["dt"])
+    if g == "normal":
+        return normal(cfg["p"], cfg["n"], cfg["seed"], cfg.get("sigma", 1.0), cfg["dt"])
+    raise ValueError(g)

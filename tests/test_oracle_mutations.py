@@ -1,0 +1,57 @@
+"""Planted mistakes: each case copies the oracle's C source, plants one
+plausible slip, builds the copy, and runs the pin tests against it.  Every
+slip must make the pins fail -- otherwise the pins could not tell a wrong
+oracle from a right one.  CPU only; the real oracle is never modified.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "rc_oracle.c")
+
+MUTANTS = {
+    "fold_starts_at_own_chunk_rank": [
+        ("int r = (int)((c + 1) % (size_t)q);", "int r = (int)(c % (size_t)q);"),
+        ("r = (int)((c + 1 + (size_t)k) % (size_t)q);", "r = (int)((c + (size_t)k) % (size_t)q);"),
+    ],
+    "fold_in_ascending_rank_order": [
+        ("int r = (int)((c + 1) % (size_t)q);", "int r = 0;"),
+        ("r = (int)((c + 1 + (size_t)k) % (size_t)q);", "r = k;"),
+    ],
+    "dropped_last_rank": [
+        ("for (int k = 1; k < q; ++k) {\n        r = (int)", "for (int k = 1; k < q - 1; ++k) {\n        r = (int)"),
+    ],
+    "sum_sign_flipped": [("acc.f = acc.f + v.f;", "acc.f = acc.f - v.f;")],
+    "max_ties_take_new_operand": [("acc.f = (v.f > acc.f) ? v.f : acc.f;", "acc.f = (v.f >= acc.f) ? v.f : acc.f;")],
+    "scale_ignored": [("float y = acc.f * scale;", "float y = acc.f;")],
+    "reduce_scatter_wrong_slice": [("size_t i = (size_t)r * m + j;", "size_t i = (size_t)((r + 1) % p) * m + j;")],
+    "bf16_ties_round_up": [("if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u) != 0u))", "if (lo >= 0x8000u)")],
+    "ring_receiver_operands_swapped": [("combine(msg[r][i - b], w[d][i], is_int, op)", "combine(w[d][i], msg[r][i - b], is_int, op)")],
+    "ring_allgather_wrong_chunk": [("size_t c = (size_t)(((r - k) % p + p) % p);", "size_t c = (size_t)(((r - k - 1) % p + p) % p);")],
+    "hier_group_drops_a_rank": [("ring_core(send + (size_t)g * (size_t)G, G,", "ring_core(send + (size_t)g * (size_t)G, G > 1 ? G - 1 : G,")],
+    "int_sum_saturates": [("acc.i = (int32_t)((uint32_t)acc.i + (uint32_t)v.i);",
+                           "{ long long t = (long long)acc.i + v.i; acc.i = t > 2147483647LL ? 2147483647 : (t < -2147483648LL ? (int32_t)-2147483648LL : (int32_t)t); }")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name):
+    src = open(SRC).read()
+    for old, new in MUTANTS[name]:
+        assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+        src = src.replace(old, new)
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "mutant.c")
+        so = os.path.join(d, "libmutant.so")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                        "-o", so, c], check=True)
+        env = dict(os.environ, RC_ORACLE_LIB=so)
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
