@@ -1,4 +1,61 @@
-"""Benchmark of the simulated-rank collectives (filled in below)."""
+"""Benchmark of librankcoll: effective GB/s of the simulated-rank collectives.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One STEP is one pass of the whole hot path over one batch of synthetic input:
+8 simulated ranks x 2,097,152 fp32 elements (8 MiB) per rank ~N(0, 1e-2),
+seed 1 (the ring / one-shot all-reduce workload), through
+  all_reduce (one-shot), reduce_scatter (fp32 -> bf16, scale 1/8),
+  all_gather (the bf16 shards), reduce (root 0), broadcast (root 0, in place),
+  ring all_reduce (literal 14 steps), hierarchical all_reduce (2 x 4, fused).
+Each collective is timed alone with CUDA events on the launching stream; an
+L2 flush (a 512 MiB write, more than the 126 MB L2) runs between collectives,
+outside the timed events, so every collective reads its inputs from HBM.
+
+Effective GB/s = minimum bytes read + written / device time (decimal GB):
+  all_reduce p*n*s_in + p*n*s_out; reduce_scatter p*n*s_in + n*s_out;
+  all_gather n*s + p*n*s; reduce p*n*s_in + n*s_out; broadcast n*s + (p-1)*n*s;
+  ring and hierarchical are charged the all_reduce minimum.
+`value` is the step's total minimum bytes over the step's total device time.
+
+`--impl reference` times the CPU oracle (single thread, host cores) on a
+bounded sample of the same workload and prints the same metric.
+With torchrun (N > 1) every rank runs its own replica of the step on its own
+GPU (no data-path collective: the simulated ranks never leave one GPU); the
+time is the max over ranks and `value` the sum of all replicas' bytes / that
+time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "effective GB/s and % of HBM peak for 8-rank all_reduce / reduce_scatter"
+UNIT = "GB/s"
+P, N = 8, 2097152
+SEED = 1
+SIGMA = 1e-2
+FLUSH_BYTES = 512 << 20
+WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 fp32 "
+            "(8 MiB) per rank ~N(0,1e-2) seed 1; step = all_reduce, reduce_scatter fp32->bf16 "
+            "x1/8, all_gather bf16, reduce, broadcast, ring all_reduce (literal), "
+            "hierarchical all_reduce 2x4 (fused)")
+
+# DRAM traffic per launch measured by ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum) for the kernel named, together with a hash of the
+# kernel's source file when it was measured; a changed source reports null.
+NCU_TRAFFIC = {}
 
 
 def busbw_all_reduce(size_bytes: float, p: int, t: float) -> float:
@@ -11,3 +68,386 @@ def busbw_reduce_scatter(input_bytes: float, p: int, t: float) -> float:
     """Bus bandwidth s_input (p-1) / (p t), same section; s_input is the
     world_size x k input of one rank."""
     return input_bytes * (p - 1) / (p * t)
+
+
+def ring_model_seconds(size_bytes: float, p: int, bw: float) -> float:
+    """Ring all-reduce time model 2 (N-1)/N * S/W ("分布式训练/推理", section
+    "Ring all-reduce 的带宽账")."""
+    return 2.0 * (p - 1) / p * size_bytes / bw
+
+
+# minimum bytes of each collective in the step (p ranks, n elements per rank)
+def step_ops(p=P, n=N):
+    s_in, s_bf = 4, 2
+    m = n // p
+    return [
+        ("all_reduce", p * n * s_in + p * n * s_in),
+        ("reduce_scatter", p * n * s_in + n * s_bf),
+        ("all_gather", n * s_bf + p * n * s_bf),
+        ("reduce", p * n * s_in + n * s_in),
+        ("broadcast", n * s_in + (p - 1) * n * s_in),
+        ("ring_all_reduce", p * n * s_in + p * n * s_in),
+        ("hier_all_reduce", p * n * s_in + p * n * s_in),
+    ], m
+
+
+KERNEL_OF = {
+    "all_reduce": ("reduce_kernel", "reduce.cu"),
+    "reduce_scatter": ("reduce_kernel", "reduce.cu"),
+    "all_gather": ("fanout_bulk_kernel", "fanout.cu"),
+    "reduce": ("reduce_kernel", "reduce.cu"),
+    "broadcast": ("fanout_bulk_kernel", "fanout.cu"),
+    "ring_all_reduce": ("ring_literal_kernel", "ring.cu"),
+    "hier_all_reduce": ("hier_fused_kernel", "hier.cu"),
+}
+
+
+def _src_hash(fname):
+    path = os.path.join(ROOT, "collective_rc_all_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"rc_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons, samples = [], [], set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                samples += 1
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    pass
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": samples}
+
+
+# ------------------------------------------------------------------ multi-rank plumbing
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def reduce_over_ranks(local_seconds: float, local_bytes: float, world: int, device=None):
+    """Max of the ranks' device times and sum of their bytes (plumbing only:
+    the timing scalars, not data).  Works with gloo (CPU) and nccl (GPU)."""
+    if world <= 1:
+        return local_seconds, local_bytes
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_seconds], dtype=torch.float64, device=device)
+    b = torch.tensor([local_bytes], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(b.item())
+
+
+# ------------------------------------------------------------------ CPU oracle arm
+def cpu_oracle_step_rate(budget_s: float = 12.0, n_sample: int = N // 8):
+    """The oracle, as it stands (one thread), on a bounded sample of the step:
+    the same seven collectives on n_sample elements per rank, repeated until
+    budget_s has passed.  Returns (GB/s, reps, seconds, n_sample)."""
+    import oracle
+    import rc_inputs
+    xs = rc_inputs.normal(P, n_sample, seed=SEED, sigma=SIGMA)
+    ops, m = step_ops(P, n_sample)
+    step_bytes = sum(b for _, b in ops)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.all_reduce(xs)
+        rs = oracle.reduce_scatter(xs, "f32", "bf16", "sum", 1.0 / P)
+        oracle.all_gather(rs, "bf16")
+        oracle.reduce(xs, 0)
+        oracle.broadcast(xs[0], P, 0)
+        oracle.ring_all_reduce(xs)
+        oracle.hier_all_reduce(xs, 4)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return step_bytes * reps / el / 1e9, reps, el, n_sample
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    ops, _ = step_ops()
+    per_step_budget = max(1.0, 20.0 / max(1, args.steps + args.warmup))
+    # warm-up steps (untimed), then K timed steps, each a bounded sample
+    for _ in range(args.warmup):
+        cpu_oracle_step_rate(budget_s=0.5 * per_step_budget)
+    rates, total_s, total_reps = [], 0.0, 0
+    for _ in range(args.steps):
+        gbs, reps, el, ns = cpu_oracle_step_rate(budget_s=per_step_budget)
+        rates.append(gbs)
+        total_s += el
+        total_reps += reps
+    value = float(np.mean(rates))
+    sample = (f"{total_reps} passes of the seven-collective step on {ns} elements per rank "
+              f"(p=8, 1/8 of the workload), one thread, {total_s:.1f} s")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "p": P, "n_per_rank": N, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+    import collective_rc_all_b200 as rc
+    import rc_inputs
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    stream = torch.cuda.current_stream()
+    ops, m = step_ops()
+    step_bytes = sum(b for _, b in ops)
+
+    # inputs: each replica draws its own batch (seed + rank)
+    xs = rc_inputs.normal(P, N, seed=SEED + rank, sigma=SIGMA)
+    send = [torch.from_numpy(x).to(dev) for x in xs]
+    f32 = lambda k: [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(k)]
+    y_ar, y_ring, y_hier = f32(P), f32(P), f32(P)
+    y_rs = [torch.empty(m, dtype=torch.bfloat16, device=dev) for _ in range(P)]
+    y_ag = [torch.empty(N, dtype=torch.bfloat16, device=dev) for _ in range(P)]
+    y_red = torch.empty(N, dtype=torch.float32, device=dev)
+    y_bc = [send[0]] + f32(P - 1)          # root 0 in place
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    cp_a = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    cp_b = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+
+    calls = {
+        "all_reduce": lambda: rc.rc_all_reduce(send, y_ar),
+        "reduce_scatter": lambda: rc.rc_reduce_scatter(send, y_rs, out_dtype="bf16", scale=1.0 / P),
+        "all_gather": lambda: rc.rc_all_gather(y_rs, y_ag),
+        "reduce": lambda: rc.rc_reduce(send, y_red, root=0),
+        "broadcast": lambda: rc.rc_broadcast(send[0], y_bc, root=0),
+        "ring_all_reduce": lambda: rc.rc_ring_all_reduce(send, y_ring, variant="literal"),
+        "hier_all_reduce": lambda: rc.rc_hier_all_reduce(send, y_hier, 4, variant="fused"),
+    }
+    names = [nm for nm, _ in ops]
+    K, W = args.steps, args.warmup
+    ev = {nm: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)] for nm in names}
+
+    def one_step(k=None):
+        for nm in names:
+            flush.zero_()                       # untimed: evicts L2 before each collective
+            if k is None:
+                calls[nm]()
+            else:
+                a, b = ev[nm][k]
+                a.record(stream)
+                calls[nm]()
+                b.record(stream)
+
+    # copy roofline of this library's own copy kernel (same run)
+    for _ in range(3):
+        rc.rc_copy(cp_a, cp_b)
+    cps = []
+    for _ in range(5):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        rc.rc_copy(cp_a, cp_b)
+        b.record(stream)
+        b.synchronize()
+        cps.append(a.elapsed_time(b) * 1e-3)
+    copy_gbs = 2 * (1 << 30) / min(cps) / 1e9
+    del cp_a, cp_b
+
+    for _ in range(W):
+        one_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    launches0 = rc.rc_launch_count()
+    for k in range(K):
+        one_step(k)
+    torch.cuda.synchronize()
+    launches = rc.rc_launch_count() - launches0
+    time.sleep(0.3)
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    rc.rc_stream_status()
+
+    per_op_s = {nm: sum(a.elapsed_time(b) for a, b in ev[nm]) * 1e-3 for nm in names}
+    local_s = sum(per_op_s.values())
+    tot_s, tot_bytes = reduce_over_ranks(local_s, step_bytes * K, world, device=dev)
+
+    # ---- end to end through the same calls with host buffers (pinned)
+    host_in = [torch.from_numpy(x).pin_memory() for x in xs]
+    outs = [y_ar[0], y_rs, y_ag[0], y_red, y_bc[1], y_ring[0], y_hier[0]]
+    flat_outs = [t for o in outs for t in (o if isinstance(o, list) else [o])]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in flat_outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    e2e_k = max(3, K // 4)
+
+    def e2e_step():
+        for d, h in zip(send, host_in):
+            d.copy_(h, non_blocking=True)
+        for nm in names:
+            calls[nm]()
+        for h, d in zip(host_out, flat_outs):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(e2e_k):
+        e2e_step()
+    eb.record(stream)
+    eb.synchronize()
+    e2e_s, e2e_bytes = reduce_over_ranks(ea.elapsed_time(eb) * 1e-3, step_bytes * e2e_k, world, device=dev)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peak, peak_kind = measured_peaks()
+    value = tot_bytes / tot_s / 1e9
+    per_op = {}
+    for nm, b in ops:
+        t = per_op_s[nm] / K
+        per_op[nm] = {"us": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
+                      "frac_of_measured_hbm": round(b / t / 1e9 / peak, 4),
+                      "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4)}
+    t_ar = per_op_s["all_reduce"] / K
+    t_rs = per_op_s["reduce_scatter"] / K
+    per_op["all_reduce"]["busbw_gib_s"] = round(busbw_all_reduce(N * 4, P, t_ar) / 2**30, 1)
+    per_op["reduce_scatter"]["busbw_gib_s"] = round(busbw_reduce_scatter(N * 4, P, t_rs) / 2**30, 1)
+    per_op["ring_all_reduce"]["ring_model_us_at_measured_hbm"] = round(
+        ring_model_seconds(N * 4, P, peak * 1e9) * 1e6, 2)
+    dom = max(names, key=lambda nm: per_op_s[nm])
+    dom_b = dict(ops)[dom]
+    dom_t = per_op_s[dom] / K
+    kname, kfile = KERNEL_OF[dom]
+    tr = NCU_TRAFFIC.get(dom)
+    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(kfile) else None
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, reps, el, ns = cpu_oracle_step_rate(budget_s=args.cpu_seconds)
+        cpu = {"value": round(gbs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{reps} passes of the seven-collective step on {ns} elements per rank "
+                         f"(p=8, 1/8 of the workload), one thread, {el:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(1e3 * tot_s / K, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "p": P, "n_per_rank": N,
+                   "l2": "flushed (512 MiB write) before every collective, outside the timed events",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": kname, "op": dom,
+                     "achieved": round(dom_b / dom_t / 1e9, 1), "peak": peak,
+                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+                     "unit": "GB/s", "frac": round(dom_b / dom_t / 1e9 / peak, 4),
+                     "traffic": traffic, "algorithmic_bytes": dom_b},
+        "per_op": per_op,
+        "copy_kernel_gbs": round(copy_gbs, 1),
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_bytes / e2e_s / 1e9, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,244 @@
+"""Python binding of librankcoll (include/rankcoll.h): collective reductions over
+p simulated ranks held in one GPU's memory.
+
+This module only marshals arguments: device pointers, sizes, enums and the
+stream go straight to the C ABI, and all work runs in the library's CUDA
+kernels.  There is no CPU fallback -- importing fails if the shared library
+has not been built (``python collective_rc_all_b200/build.py``).
+
+Each ``rc_*`` function mirrors the C entry point of the same name.  Buffers
+may be given as CUDA tensors (contiguous) or as integer device addresses; for
+tensors, ``n`` and ``dtype`` default to what the tensors say.  ``stream``
+defaults to torch's current stream.  A non-OK status raises RankCollError
+carrying the library's message.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Union
+
+__all__ = [
+    "RankCollError", "lib", "library_path",
+    "FP32", "BF16", "INT32", "SUM", "MAX", "MIN", "RING_LITERAL", "RING_ONESHOT",
+    "HIER_FUSED", "HIER_STAGED",
+    "rc_all_reduce", "rc_reduce_scatter", "rc_all_gather", "rc_reduce", "rc_broadcast",
+    "rc_ring_all_reduce", "rc_hier_all_reduce", "rc_copy", "rc_reserve_workspace", "rc_check_buffer",
+    "rc_stream_status", "rc_launch_count", "rc_finalize", "rc_version", "rc_last_error",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "librankcoll.so")
+
+if not os.path.exists(library_path):
+    raise ImportError(
+        f"librankcoll.so not found at {library_path}; build it with "
+        "`python collective_rc_all_b200/build.py` (there is no CPU fallback)")
+
+lib = ctypes.CDLL(library_path)
+
+# enums (values fixed by include/rankcoll.h)
+FP32, BF16, INT32 = 0, 1, 2
+SUM, MAX, MIN = 0, 1, 2
+RING_LITERAL, RING_ONESHOT = 0, 1
+HIER_FUSED, HIER_STAGED = 0, 1
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "timeout"}
+
+_vpp = ctypes.POINTER(ctypes.c_void_p)
+_sz, _i, _f, _vp = ctypes.c_size_t, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+
+
+def _decl(name, args, res=ctypes.c_int):
+    fn = getattr(lib, name)
+    fn.argtypes = args
+    fn.restype = res
+    return fn
+
+
+_decl("rc_all_reduce", [_vpp, _vpp, _i, _sz, _i, _i, _f, _vp])
+_decl("rc_reduce_scatter", [_vpp, _vpp, _i, _sz, _i, _i, _i, _f, _vp])
+_decl("rc_all_gather", [_vpp, _vpp, _i, _sz, _i, _vp])
+_decl("rc_reduce", [_vpp, _vp, _i, _i, _sz, _i, _i, _f, _vp])
+_decl("rc_broadcast", [_vp, _vpp, _i, _i, _sz, _i, _vp])
+_decl("rc_ring_all_reduce", [_vpp, _vpp, _i, _sz, _i, _i, _f, _i, _vp])
+_decl("rc_hier_all_reduce", [_vpp, _vpp, _i, _i, _sz, _i, _i, _f, _i, _vp])
+_decl("rc_copy", [_vp, _vp, _sz, _vp])
+_decl("rc_reserve_workspace", [_sz, _vp])
+_decl("rc_check_buffer", [_vp, _sz])
+_decl("rc_stream_status", [_vp])
+_decl("rc_status_string", [_i], ctypes.c_char_p)
+_decl("rc_last_error", [], ctypes.c_char_p)
+_decl("rc_launch_count", [], ctypes.c_uint64)
+_decl("rc_finalize", [])
+_decl("rc_version", [])
+
+
+class RankCollError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.rc_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {_STATUS.get(status, status)}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise RankCollError(status, where)
+
+
+# ---------------------------------------------------------------- marshalling
+_DT_NAMES = {"f32": FP32, "fp32": FP32, "float32": FP32, "bf16": BF16, "bfloat16": BF16,
+             "i32": INT32, "int32": INT32}
+_OP_NAMES = {"sum": SUM, "max": MAX, "min": MIN}
+
+
+def _is_tensor(x) -> bool:
+    return hasattr(x, "data_ptr") and hasattr(x, "dtype")
+
+
+def _dt(dtype, like=None) -> int:
+    if dtype is None:
+        if like is None or not _is_tensor(like):
+            raise ValueError("dtype is required when buffers are raw addresses")
+        import torch
+        m = {torch.float32: FP32, torch.bfloat16: BF16, torch.int32: INT32}
+        if like.dtype not in m:
+            raise TypeError(f"unsupported tensor dtype {like.dtype}")
+        return m[like.dtype]
+    if isinstance(dtype, str):
+        return _DT_NAMES[dtype.lower()]
+    if isinstance(dtype, int):
+        return dtype
+    import torch
+    return {torch.float32: FP32, torch.bfloat16: BF16, torch.int32: INT32}[dtype]
+
+
+def _op(op) -> int:
+    return _OP_NAMES[op.lower()] if isinstance(op, str) else int(op)
+
+
+def _addr(x) -> int:
+    if _is_tensor(x):
+        if not x.is_cuda:
+            raise ValueError("tensor is not on a CUDA device")
+        if not x.is_contiguous():
+            raise ValueError("tensor must be contiguous")
+        return x.data_ptr()
+    return int(x)
+
+
+def _ptrs(xs: Sequence) -> "ctypes.Array":
+    return (ctypes.c_void_p * len(xs))(*[_addr(x) for x in xs])
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if hasattr(stream, "cuda_stream"):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _numel(x, n):
+    if n is not None:
+        return int(n)
+    if _is_tensor(x):
+        return x.numel()
+    raise ValueError("n is required when buffers are raw addresses")
+
+
+Buf = Union[int, "torch.Tensor"]  # noqa: F821
+
+
+# ---------------------------------------------------------------- entry points
+def rc_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], n=None, dtype=None, op="sum",
+                  scale=1.0, stream=None):
+    p = len(send)
+    _check(lib.rc_all_reduce(_ptrs(send), _ptrs(recv), p, _numel(send[0], n), _dt(dtype, send[0]),
+                             _op(op), scale, _stream(stream)), "rc_all_reduce")
+
+
+def rc_reduce_scatter(send: Sequence[Buf], recv: Sequence[Buf], n=None, in_dtype=None,
+                      out_dtype=None, op="sum", scale=1.0, stream=None):
+    p = len(send)
+    _check(lib.rc_reduce_scatter(_ptrs(send), _ptrs(recv), p, _numel(send[0], n),
+                                 _dt(in_dtype, send[0]), _dt(out_dtype, recv[0]), _op(op), scale,
+                                 _stream(stream)), "rc_reduce_scatter")
+
+
+def rc_all_gather(send: Sequence[Buf], recv: Sequence[Buf], n=None, dtype=None, stream=None):
+    p = len(send)
+    nn = int(n) if n is not None else _numel(recv[0], None)
+    _check(lib.rc_all_gather(_ptrs(send), _ptrs(recv), p, nn, _dt(dtype, send[0]), _stream(stream)),
+           "rc_all_gather")
+
+
+def rc_reduce(send: Sequence[Buf], recv_root: Buf, root=0, n=None, dtype=None, op="sum",
+              scale=1.0, stream=None):
+    p = len(send)
+    _check(lib.rc_reduce(_ptrs(send), _addr(recv_root), p, root, _numel(send[0], n),
+                         _dt(dtype, send[0]), _op(op), scale, _stream(stream)), "rc_reduce")
+
+
+def rc_broadcast(send_root: Buf, recv: Sequence[Buf], root=0, n=None, dtype=None, stream=None):
+    p = len(recv)
+    _check(lib.rc_broadcast(_addr(send_root), _ptrs(recv), p, root, _numel(send_root, n),
+                            _dt(dtype, send_root), _stream(stream)), "rc_broadcast")
+
+
+def rc_ring_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], n=None, dtype=None, op="sum",
+                       scale=1.0, variant=RING_LITERAL, stream=None):
+    p = len(send)
+    v = {"literal": RING_LITERAL, "oneshot": RING_ONESHOT}.get(variant, variant)
+    _check(lib.rc_ring_all_reduce(_ptrs(send), _ptrs(recv), p, _numel(send[0], n),
+                                  _dt(dtype, send[0]), _op(op), scale, int(v), _stream(stream)),
+           "rc_ring_all_reduce")
+
+
+def rc_hier_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], group_size: int, n=None,
+                       dtype=None, op="sum", scale=1.0, variant=HIER_FUSED, stream=None):
+    p = len(send)
+    v = {"fused": HIER_FUSED, "staged": HIER_STAGED}.get(variant, variant)
+    _check(lib.rc_hier_all_reduce(_ptrs(send), _ptrs(recv), p, group_size, _numel(send[0], n),
+                                  _dt(dtype, send[0]), _op(op), scale, int(v), _stream(stream)),
+           "rc_hier_all_reduce")
+
+
+def rc_copy(src: Buf, dst: Buf, nbytes=None, stream=None):
+    if nbytes is None:
+        nbytes = src.numel() * src.element_size()
+    _check(lib.rc_copy(_addr(src), _addr(dst), int(nbytes), _stream(stream)), "rc_copy")
+
+
+def rc_check_buffer(buf: Buf, nbytes: int) -> None:
+    """Raise unless [buf, buf + nbytes) is device memory of the current device
+    inside one allocation (no launch)."""
+    _check(lib.rc_check_buffer(_addr(buf), int(nbytes)), "rc_check_buffer")
+
+
+def rc_reserve_workspace(nbytes: int, stream=None):
+    _check(lib.rc_reserve_workspace(int(nbytes), _stream(stream)), "rc_reserve_workspace")
+
+
+def rc_stream_status(stream=None) -> int:
+    """Synchronise the stream; raise on an asynchronous error or a device wait
+    that gave up; return 0 otherwise."""
+    st = lib.rc_stream_status(_stream(stream))
+    _check(st, "rc_stream_status")
+    return st
+
+
+def rc_launch_count() -> int:
+    return int(lib.rc_launch_count())
+
+
+def rc_finalize():
+    _check(lib.rc_finalize(), "rc_finalize")
+
+
+def rc_version() -> int:
+    return int(lib.rc_version())
+
+
+def rc_last_error() -> str:
+    return lib.rc_last_error().decode(errors="replace")

@@ -1,0 +1,554 @@
+// api.cu -- the extern "C" entry points of librankcoll (include/rankcoll.h):
+// argument validation, aliasing rules, workspace management, dispatch.
+//
+// Every check happens on the host before anything is enqueued, so a bad call
+// returns an error code and never reaches the GPU.  Device pointers are
+// checked against the allocation that contains them (driver address-range
+// query): a host pointer, a pointer from another device, or a buffer too small
+// for the requested elements is RC_ERR_INVALID_ARG.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/rankcoll.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace rc {
+
+// ---------------------------------------------------------------- bookkeeping
+namespace {
+thread_local char t_last_error[512] = "";
+std::atomic<uint64_t> g_launches{0};
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+rc_status fail(rc_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+rc_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(RC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int v = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_sm_count[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+void note_launches(int k) { g_launches.fetch_add((uint64_t)k, std::memory_order_relaxed); }
+
+int env_int(const char *name, int dflt) {
+  const char *v = getenv(name);
+  if (!v || !*v) return dflt;
+  return atoi(v);
+}
+
+// ---------------------------------------------------------------- pointer checks
+namespace {
+
+typedef CUresult (*MemGetAddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+MemGetAddressRangeFn address_range_fn() {
+  static MemGetAddressRangeFn fn = []() -> MemGetAddressRangeFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<MemGetAddressRangeFn>(p);
+  }();
+  return fn;
+}
+
+// [ptr, ptr+bytes) must be device (or managed) memory of the current device,
+// inside one allocation.
+rc_status check_device_range(const void *ptr, size_t bytes, const char *what, int idx) {
+  if (ptr == nullptr) return fail(RC_ERR_INVALID_ARG, "%s[%d] is NULL", what, idx);
+  cudaPointerAttributes at{};
+  cudaError_t e = cudaPointerGetAttributes(&at, ptr);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p is not a CUDA pointer (%s)", what, idx, ptr,
+                cudaGetErrorString(e));
+  }
+  if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+    return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p is not device memory", what, idx, ptr);
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (at.type == cudaMemoryTypeDevice && at.device != dev)
+    return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p lives on device %d, current device is %d", what, idx,
+                ptr, at.device, dev);
+  if (env_int("RC_SKIP_RANGE_CHECK", 0)) return RC_OK;
+  MemGetAddressRangeFn fn = address_range_fn();
+  if (fn) {
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (fn(&base, &size, (CUdeviceptr)(uintptr_t)ptr) == CUDA_SUCCESS) {
+      const uintptr_t p = (uintptr_t)ptr;
+      if (p < (uintptr_t)base || p - (uintptr_t)base > size || bytes > size - (p - (uintptr_t)base))
+        return fail(RC_ERR_INVALID_ARG,
+                    "%s[%d]=%p: %zu bytes run past the end of its allocation (%zu bytes at %p)", what,
+                    idx, ptr, bytes, size, (void *)base);
+    }
+  }
+  return RC_OK;
+}
+
+struct Buf {
+  uintptr_t lo, hi;   // byte range
+  intptr_t origin;    // address of global element 0 under this buffer's indexing
+  int esz;
+  int rank;
+  bool out;
+  const char *what;
+  int idx;
+};
+
+Buf make_buf(const void *p, uint64_t elems, int esz, uint64_t index0, int rank, bool out,
+             const char *what, int idx) {
+  Buf b;
+  b.lo = (uintptr_t)p;
+  b.hi = b.lo + elems * (uint64_t)esz;
+  b.origin = (intptr_t)(b.lo - index0 * (uint64_t)esz);
+  b.esz = esz;
+  b.rank = rank;
+  b.out = out;
+  b.what = what;
+  b.idx = idx;
+  return b;
+}
+
+// Outputs must not overlap each other; an output may overlap an input only if
+// both belong to the same rank and address the same elements identically.
+rc_status check_aliasing(const std::vector<Buf> &bs) {
+  for (size_t i = 0; i < bs.size(); ++i) {
+    for (size_t j = i + 1; j < bs.size(); ++j) {
+      const Buf &a = bs[i], &b = bs[j];
+      if (!a.out && !b.out) continue;
+      if (a.lo >= b.hi || b.lo >= a.hi || a.lo == a.hi || b.lo == b.hi) continue;
+      if (a.out && b.out)
+        return fail(RC_ERR_INVALID_ARG, "output buffers %s[%d] and %s[%d] overlap", a.what, a.idx,
+                    b.what, b.idx);
+      if (a.rank != b.rank || a.esz != b.esz || a.origin != b.origin)
+        return fail(RC_ERR_INVALID_ARG,
+                    "%s[%d] and %s[%d] overlap in a way other than same-rank in-place", a.what,
+                    a.idx, b.what, b.idx);
+    }
+  }
+  return RC_OK;
+}
+
+rc_status check_ranges(const std::vector<Buf> &bs) {
+  for (const Buf &b : bs) {
+    rc_status st = check_device_range((const void *)b.lo, b.hi - b.lo, b.what, b.idx);
+    if (st != RC_OK) return st;
+  }
+  return RC_OK;
+}
+
+int dt_size(rc_dtype d) { return d == RC_BF16 ? 2 : 4; }
+bool dt_ok(int d) { return d == RC_FP32 || d == RC_BF16 || d == RC_INT32; }
+bool op_ok(int o) { return o == RC_SUM || o == RC_MAX || o == RC_MIN; }
+
+constexpr uint64_t kMaxElems = (1ull << 40);  // 1 Ti elements per rank
+
+rc_status check_p_n(int p, size_t n) {
+  if (p < 1 || p > kMaxP) return fail(RC_ERR_INVALID_ARG, "p=%d outside [1, %d]", p, kMaxP);
+  if (n > kMaxElems) return fail(RC_ERR_INVALID_ARG, "n=%zu too large", n);
+  return RC_OK;
+}
+
+rc_status check_reduce_types(rc_dtype in, rc_dtype out, rc_op op, float scale) {
+  if (!dt_ok(in) || !dt_ok(out)) return fail(RC_ERR_INVALID_ARG, "unknown dtype");
+  if (!op_ok(op)) return fail(RC_ERR_INVALID_ARG, "unknown op");
+  if ((in == RC_INT32) != (out == RC_INT32))
+    return fail(RC_ERR_INVALID_ARG, "int32 reduces only to int32");
+  if ((in == RC_INT32 || op != RC_SUM) && scale != 1.0f)
+    return fail(RC_ERR_INVALID_ARG, "scale must be 1 unless op is SUM on a floating type");
+  return RC_OK;
+}
+
+rc_status launched(cudaError_t e, const char *what) {
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return RC_OK;
+}
+
+// ---------------------------------------------------------------- workspace
+// One workspace per device.  A call on a stream other than the last user's
+// first waits for the last user's work (event), so concurrent streams never
+// share it; growth frees the old block in stream order.
+struct Workspace {
+  void *ptr = nullptr;
+  size_t cap = 0;
+  cudaStream_t last = nullptr;
+  cudaEvent_t done = nullptr;
+  bool used = false;
+};
+std::mutex g_ws_mu;
+Workspace g_ws[kMaxDevices];
+
+rc_status ws_acquire(size_t bytes, cudaStream_t s, void **out, int *dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(RC_ERR_UNSUPPORTED, "device index %d", dev);
+  Workspace &w = g_ws[dev];
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cap);
+  if (cap != cudaStreamCaptureStatusNone) {
+    if (w.cap < bytes)
+      return fail(RC_ERR_INVALID_ARG,
+                  "workspace of %zu bytes needed during stream capture: call "
+                  "rc_reserve_workspace first",
+                  bytes);
+    *out = w.ptr;
+    *dev_out = -1;  // no event bookkeeping inside a capture
+    return RC_OK;
+  }
+  if (!w.done) {
+    if ((e = cudaEventCreateWithFlags(&w.done, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "cudaEventCreate");
+  }
+  if (w.used && w.last != s) {
+    if ((e = cudaStreamWaitEvent(s, w.done, 0)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamWaitEvent");
+  }
+  if (w.cap < bytes) {
+    if (w.ptr) {
+      if ((e = cudaFreeAsync(w.ptr, s)) != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+      w.ptr = nullptr;
+      w.cap = 0;
+    }
+    const size_t want = (bytes + 255) & ~(size_t)255;
+    if ((e = cudaMallocAsync(&w.ptr, want, s)) != cudaSuccess) {
+      w.ptr = nullptr;
+      return cuda_fail(e, "cudaMallocAsync(workspace)");
+    }
+    w.cap = want;
+  }
+  *out = w.ptr;
+  *dev_out = dev;
+  return RC_OK;
+}
+
+void ws_release(int dev, cudaStream_t s) {
+  if (dev < 0) return;
+  Workspace &w = g_ws[dev];
+  cudaEventRecord(w.done, s);
+  w.last = s;
+  w.used = true;
+}
+
+}  // namespace
+}  // namespace rc
+
+using namespace rc;
+
+extern "C" {
+
+rc_status rc_all_reduce(const void *const *send, void *const *recv, int p, size_t n, rc_dtype dt,
+                        rc_op op, float scale, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(dt, dt, op, scale)) != RC_OK) return st;
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, s, 0, r, false, "send", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  ReduceJob j{};
+  j.p = p;
+  j.n = n;
+  for (int r = 0; r < p; ++r) {
+    j.src[r] = send[r];
+    j.dst[r] = recv[r];
+  }
+  j.in_dt = j.out_dt = dt;
+  j.op = op;
+  j.scale = scale;
+  j.mode = kModeAll;
+  j.ndst = p;
+  return launched(launch_reduce(j, (cudaStream_t)stream), "all_reduce launch");
+}
+
+rc_status rc_reduce_scatter(const void *const *send, void *const *recv, int p, size_t n,
+                            rc_dtype in_dt, rc_dtype out_dt, rc_op op, float scale,
+                            rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(in_dt, out_dt, op, scale)) != RC_OK) return st;
+  if (n % (size_t)p != 0) return fail(RC_ERR_INVALID_ARG, "n=%zu is not a multiple of p=%d", n, p);
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const uint64_t m = n / p;
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, dt_size(in_dt), 0, r, false, "send", r));
+  for (int r = 0; r < p; ++r)
+    bs.push_back(make_buf(recv[r], m, dt_size(out_dt), (uint64_t)r * m, r, true, "recv", r));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  ReduceJob j{};
+  j.p = p;
+  j.n = n;
+  for (int r = 0; r < p; ++r) {
+    j.src[r] = send[r];
+    j.dst[r] = recv[r];
+  }
+  j.in_dt = in_dt;
+  j.out_dt = out_dt;
+  j.op = op;
+  j.scale = scale;
+  j.mode = kModeScatter;
+  return launched(launch_reduce(j, (cudaStream_t)stream), "reduce_scatter launch");
+}
+
+rc_status rc_all_gather(const void *const *send, void *const *recv, int p, size_t n, rc_dtype dt,
+                        rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if (!dt_ok(dt)) return fail(RC_ERR_INVALID_ARG, "unknown dtype");
+  if (n % (size_t)p != 0) return fail(RC_ERR_INVALID_ARG, "n=%zu is not a multiple of p=%d", n, p);
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  const uint64_t m = n / p;
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], m, s, (uint64_t)r * m, r, false, "send", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  FanoutJob f{};
+  f.nsrc = p;
+  f.p = p;
+  f.src_bytes = m * s;
+  f.elem_bytes = s;
+  for (int r = 0; r < p; ++r) {
+    f.src[r] = send[r];
+    f.dst[r] = recv[r];
+  }
+  for (int q = 0; q < p; ++q)
+    for (int r = 0; r < p; ++r)
+      if ((const char *)recv[q] + (uint64_t)r * m * s == (const char *)send[r]) f.skip[q] |= 1u << r;
+  return launched(launch_fanout(f, (cudaStream_t)stream), "all_gather launch");
+}
+
+rc_status rc_reduce(const void *const *send, void *recv_root, int p, int root, size_t n, rc_dtype dt,
+                    rc_op op, float scale, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(dt, dt, op, scale)) != RC_OK) return st;
+  if (root < 0 || root >= p) return fail(RC_ERR_INVALID_ARG, "root=%d outside [0, %d)", root, p);
+  if (n == 0) return RC_OK;
+  if (!send) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, s, 0, r, false, "send", r));
+  bs.push_back(make_buf(recv_root, n, s, 0, root, true, "recv_root", 0));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  ReduceJob j{};
+  j.p = p;
+  j.n = n;
+  for (int r = 0; r < p; ++r) j.src[r] = send[r];
+  j.dst[0] = recv_root;
+  j.in_dt = j.out_dt = dt;
+  j.op = op;
+  j.scale = scale;
+  j.mode = kModeOne;
+  return launched(launch_reduce(j, (cudaStream_t)stream), "reduce launch");
+}
+
+rc_status rc_broadcast(const void *send_root, void *const *recv, int p, int root, size_t n,
+                       rc_dtype dt, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if (!dt_ok(dt)) return fail(RC_ERR_INVALID_ARG, "unknown dtype");
+  if (root < 0 || root >= p) return fail(RC_ERR_INVALID_ARG, "root=%d outside [0, %d)", root, p);
+  if (n == 0) return RC_OK;
+  if (!recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  bs.push_back(make_buf(send_root, n, s, 0, root, false, "send_root", 0));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  FanoutJob f{};
+  f.nsrc = 1;
+  f.p = p;
+  f.src_bytes = (uint64_t)n * s;
+  f.elem_bytes = s;
+  f.src[0] = send_root;
+  for (int q = 0; q < p; ++q) {
+    f.dst[q] = recv[q];
+    if (recv[q] == send_root) f.skip[q] = 1u;
+  }
+  return launched(launch_fanout(f, (cudaStream_t)stream), "broadcast launch");
+}
+
+rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, size_t n, rc_dtype dt,
+                             rc_op op, float scale, rc_ring_variant variant, rc_stream_t stream) {
+  if (variant == RC_RING_ONESHOT) return rc_all_reduce(send, recv, p, n, dt, op, scale, stream);
+  if (variant != RC_RING_LITERAL) return fail(RC_ERR_INVALID_ARG, "unknown ring variant");
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(dt, dt, op, scale)) != RC_OK) return st;
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  if (p == 1) return rc_all_reduce(send, recv, p, n, dt, op, scale, stream);  // no steps
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, s, 0, r, false, "send", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  RingJob j{};
+  j.p = p;
+  j.n = n;
+  j.dt = dt;
+  j.op = op;
+  j.scale = scale;
+  for (int r = 0; r < p; ++r) {
+    j.x[r] = send[r];
+    j.y[r] = recv[r];
+  }
+  int dev = -1;
+  const uint64_t C = (n + p - 1) / p;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  if (dt == RC_BF16) {
+    if ((st = ws_acquire(2ull * p * C * 4, (cudaStream_t)stream, &j.ws, &dev)) != RC_OK) return st;
+  }
+  st = launched(launch_ring_literal(j, (cudaStream_t)stream), "ring launch");
+  if (dt == RC_BF16) ws_release(dev, (cudaStream_t)stream);
+  return st;
+}
+
+rc_status rc_hier_all_reduce(const void *const *send, void *const *recv, int p, int group_size,
+                             size_t n, rc_dtype dt, rc_op op, float scale, rc_hier_variant variant,
+                             rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(dt, dt, op, scale)) != RC_OK) return st;
+  if (group_size < 1 || p % group_size != 0)
+    return fail(RC_ERR_INVALID_ARG, "group_size=%d does not divide p=%d", group_size, p);
+  if (variant != RC_HIER_FUSED && variant != RC_HIER_STAGED)
+    return fail(RC_ERR_INVALID_ARG, "unknown hierarchical variant");
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, s, 0, r, false, "send", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  HierJob j{};
+  j.p = p;
+  j.G = group_size;
+  j.n = n;
+  j.dt = dt;
+  j.op = op;
+  j.scale = scale;
+  for (int r = 0; r < p; ++r) {
+    j.x[r] = send[r];
+    j.y[r] = recv[r];
+  }
+  if (variant == RC_HIER_FUSED) return launched(launch_hier_fused(j, (cudaStream_t)stream), "hier launch");
+  int dev = -1;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  const uint64_t ng = (uint64_t)(p / group_size);
+  if ((st = ws_acquire((ng + 1) * n * 4, (cudaStream_t)stream, &j.ws, &dev)) != RC_OK) return st;
+  st = launched(launch_hier_staged(j, (cudaStream_t)stream), "hier staged launch");
+  ws_release(dev, (cudaStream_t)stream);
+  return st;
+}
+
+rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream) {
+  if (bytes == 0) return RC_OK;
+  rc_status st;
+  if ((st = check_device_range(src, bytes, "src", 0)) != RC_OK) return st;
+  if ((st = check_device_range(dst, bytes, "dst", 0)) != RC_OK) return st;
+  const uintptr_t a = (uintptr_t)src, b = (uintptr_t)dst;
+  if (a < b + bytes && b < a + bytes) return fail(RC_ERR_INVALID_ARG, "src and dst overlap");
+  return launched(launch_copy(src, dst, bytes, (cudaStream_t)stream), "copy launch");
+}
+
+rc_status rc_check_buffer(const void *ptr, size_t bytes) {
+  return check_device_range(ptr, bytes, "buffer", 0);
+}
+
+rc_status rc_reserve_workspace(size_t bytes, rc_stream_t stream) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  void *p = nullptr;
+  int dev = -1;
+  rc_status st = ws_acquire(bytes, (cudaStream_t)stream, &p, &dev);
+  if (st == RC_OK) ws_release(dev, (cudaStream_t)stream);
+  return st;
+}
+
+rc_status rc_stream_status(rc_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream");
+  unsigned int timeouts = 0;
+  e = read_and_clear_wait_timeouts(&timeouts);
+  if (e != cudaSuccess) return cuda_fail(e, "status word");
+  if (timeouts) return fail(RC_ERR_TIMEOUT, "%u bounded device wait(s) gave up", timeouts);
+  return RC_OK;
+}
+
+const char *rc_status_string(rc_status s) {
+  switch (s) {
+    case RC_OK: return "ok";
+    case RC_ERR_INVALID_ARG: return "invalid argument";
+    case RC_ERR_UNSUPPORTED: return "unsupported";
+    case RC_ERR_CUDA: return "CUDA error";
+    case RC_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char *rc_last_error(void) { return t_last_error; }
+
+uint64_t rc_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+rc_status rc_finalize(void) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  rc_status st = RC_OK;
+  for (int d = 0; d < kMaxDevices; ++d) {
+    Workspace &w = g_ws[d];
+    if (!w.ptr && !w.done) continue;
+    cudaSetDevice(d);
+    cudaDeviceSynchronize();
+    if (w.ptr && cudaFree(w.ptr) != cudaSuccess) st = fail(RC_ERR_CUDA, "cudaFree(workspace)");
+    if (w.done) cudaEventDestroy(w.done);
+    w = Workspace{};
+  }
+  cudaSetDevice(cur);
+  return st;
+}
+
+int rc_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,204 @@
+// common.cuh -- device helpers shared by the librankcoll kernels (sm_100a).
+//
+// Arithmetic contract of every reducing kernel (see include/rankcoll.h):
+// fp32 accumulate with IEEE round-to-nearest-even adds (the library is built
+// with -fmad=false and without fast-math, so no contraction and no flush to
+// zero), compare-select MAX/MIN, wrapping int32 adds, one fp32 multiply by
+// `scale` after the fold, bf16 narrowing with the round-to-nearest-even
+// conversion intrinsics.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace rc {
+
+enum Dtype : int { kF32 = 0, kBF16 = 1, kI32 = 2 };
+enum Op : int { kSum = 0, kMax = 1, kMin = 2 };
+
+constexpr int kMaxRanks = 16;
+
+// ---------------------------------------------------------------- type traits
+// Storage tags.  Each has: bytes per element, the accumulator type, and
+// widen / narrow conversions.
+struct F32 {
+  static constexpr int kBytes = 4;
+  using Acc = float;
+};
+struct BF16 {
+  static constexpr int kBytes = 2;
+  using Acc = float;
+};
+struct I32 {
+  static constexpr int kBytes = 4;
+  using Acc = int32_t;
+};
+
+// ---------------------------------------------------------------- reductions
+template <int OP>
+__device__ __forceinline__ float combine(float acc, float v) {
+  if constexpr (OP == kSum) {
+    return __fadd_rn(acc, v);
+  } else if constexpr (OP == kMax) {
+    return (v > acc) ? v : acc;
+  } else {
+    return (v < acc) ? v : acc;
+  }
+}
+
+template <int OP>
+__device__ __forceinline__ int32_t combine(int32_t acc, int32_t v) {
+  if constexpr (OP == kSum) {
+    return (int32_t)((uint32_t)acc + (uint32_t)v);
+  } else if constexpr (OP == kMax) {
+    return (v > acc) ? v : acc;
+  } else {
+    return (v < acc) ? v : acc;
+  }
+}
+
+// One multiply by scale for floating SUM; other ops carry scale == 1 and the
+// value is passed through unchanged.
+template <int OP>
+__device__ __forceinline__ float finish(float acc, float scale) {
+  if constexpr (OP == kSum) {
+    return __fmul_rn(acc, scale);
+  } else {
+    return acc;
+  }
+}
+template <int OP>
+__device__ __forceinline__ int32_t finish(int32_t acc, float) {
+  return acc;
+}
+
+// ---------------------------------------------------------------- conversions
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h16) {
+  return __uint_as_float(h16 << 16);
+}
+
+// two fp32 -> packed bf16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Scalar element load/store in a storage type, widened to the accumulator.
+template <class T>
+__device__ __forceinline__ typename T::Acc load_elem(const char *base, uint64_t i);
+template <>
+__device__ __forceinline__ float load_elem<F32>(const char *base, uint64_t i) {
+  return reinterpret_cast<const float *>(base)[i];
+}
+template <>
+__device__ __forceinline__ float load_elem<BF16>(const char *base, uint64_t i) {
+  return bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(base)[i]);
+}
+template <>
+__device__ __forceinline__ int32_t load_elem<I32>(const char *base, uint64_t i) {
+  return reinterpret_cast<const int32_t *>(base)[i];
+}
+
+template <class T>
+__device__ __forceinline__ void store_elem(char *base, uint64_t i, typename T::Acc v);
+template <>
+__device__ __forceinline__ void store_elem<F32>(char *base, uint64_t i, float v) {
+  reinterpret_cast<float *>(base)[i] = v;
+}
+template <>
+__device__ __forceinline__ void store_elem<BF16>(char *base, uint64_t i, float v) {
+  reinterpret_cast<uint16_t *>(base)[i] = f32_to_bf16_bits(v);
+}
+template <>
+__device__ __forceinline__ void store_elem<I32>(char *base, uint64_t i, int32_t v) {
+  reinterpret_cast<int32_t *>(base)[i] = v;
+}
+
+// ---------------------------------------------------------------- 16-byte vectors
+// A 16-byte vector of input type T holds kVec<T> elements.
+template <class T>
+constexpr int kVec = 16 / T::kBytes;
+
+// Read-only streaming load: non-coherent path, no L1 allocation.  Only for
+// data no thread writes before this thread's own read of it in the kernel.
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_v4(void *p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_v2(void *p, uint2 v) {
+  asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// Unpack a raw 16-byte vector of T into kVec<T> accumulators.
+template <class T>
+__device__ __forceinline__ void unpack(const uint4 &raw, typename T::Acc (&a)[kVec<T>]);
+template <>
+__device__ __forceinline__ void unpack<F32>(const uint4 &raw, float (&a)[4]) {
+  a[0] = __uint_as_float(raw.x);
+  a[1] = __uint_as_float(raw.y);
+  a[2] = __uint_as_float(raw.z);
+  a[3] = __uint_as_float(raw.w);
+}
+template <>
+__device__ __forceinline__ void unpack<I32>(const uint4 &raw, int32_t (&a)[4]) {
+  a[0] = (int32_t)raw.x;
+  a[1] = (int32_t)raw.y;
+  a[2] = (int32_t)raw.z;
+  a[3] = (int32_t)raw.w;
+}
+template <>
+__device__ __forceinline__ void unpack<BF16>(const uint4 &raw, float (&a)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    a[2 * j] = __uint_as_float(w[j] << 16);
+    a[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+  }
+}
+
+// Store VEC accumulated values (already scaled) as type TO at address p.
+// VEC * TO::kBytes is 8, 16 or 32 bytes.
+template <class TO, int VEC>
+__device__ __forceinline__ void store_vec(char *p, const typename TO::Acc (&y)[VEC]);
+
+template <>
+__device__ __forceinline__ void store_vec<F32, 4>(char *p, const float (&y)[4]) {
+  st_v4(p, make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                      __float_as_uint(y[3])));
+}
+template <>
+__device__ __forceinline__ void store_vec<I32, 4>(char *p, const int32_t (&y)[4]) {
+  st_v4(p, make_uint4((uint32_t)y[0], (uint32_t)y[1], (uint32_t)y[2], (uint32_t)y[3]));
+}
+template <>
+__device__ __forceinline__ void store_vec<BF16, 8>(char *p, const float (&y)[8]) {
+  st_v4(p, make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                      pack_bf16x2(y[6], y[7])));
+}
+template <>
+__device__ __forceinline__ void store_vec<BF16, 4>(char *p, const float (&y)[4]) {
+  st_v2(p, make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3])));
+}
+template <>
+__device__ __forceinline__ void store_vec<F32, 8>(char *p, const float (&y)[8]) {
+  st_v4(p, make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                      __float_as_uint(y[3])));
+  st_v4(p + 16, make_uint4(__float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]),
+                           __float_as_uint(y[7])));
+}
+
+}  // namespace rc

@@ -1,0 +1,184 @@
+// fanout.cu -- all-gather and broadcast as a bulk-copy fan-out.
+//
+// Pages: "分布式训练/推理", section "通信原语：rank、world size 和 collective
+// operations" (broadcast copies one rank's tensor to every rank; all-gather
+// hands every rank the concatenation of all shards) and section
+// "FSDP 的执行顺序" (parameter shards all-gathered before the module runs).
+//
+// Each source tile is read from HBM ONCE into the CTA's own shared memory by
+// a bulk copy (TMA engine, completion on an mbarrier) and written out p times
+// by bulk stores -- minimum traffic n*s read + p*n*s written.  One elected
+// thread per CTA drives a STAGES-deep ring of shared-memory tiles: loads run
+// LOOKAHEAD tiles ahead of the stores, and a stage is refilled only after the
+// stores that read it have finished reading (bulk wait_group.read).  Plain
+// (non-multicast) copies only: every load targets this CTA's own shared
+// memory from this GPU's own memory.
+//
+// Every wait is bounded (2 s on the global timer).  On expiry the kernel
+// counts the event in a device word, drains its own copies (again bounded)
+// and returns; rc_stream_status() reports RC_ERR_TIMEOUT.
+#include <algorithm>
+#include <atomic>
+
+#include "bulk.cuh"
+#include "common.cuh"
+#include "internal.h"
+
+namespace rc {
+
+// Number of bounded waits that gave up since the host last looked.
+__device__ unsigned int g_wait_timeouts = 0;
+
+namespace {
+
+constexpr uint32_t kTile = 32 * 1024;  // bytes per stage
+constexpr int kStages = 6;
+constexpr int kLookahead = 4;          // loads in flight ahead of the stores
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+static_assert(kLookahead <= kStages - 1, "a stage must be free when its load is issued");
+
+struct FanoutParams {
+  const char *src[kMaxRanks];
+  char *dst[kMaxRanks];
+  uint32_t skip[kMaxRanks];  // bit r of skip[q]: do not write source r to rank q
+  uint64_t src_bytes;
+  uint64_t tiles_per_src;
+  uint64_t units;            // nsrc * tiles_per_src
+  int p;
+};
+
+__global__ void __launch_bounds__(32) fanout_bulk_kernel(const __grid_constant__ FanoutParams a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bars[kStages];
+  if (threadIdx.x != 0) return;
+
+  for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+  mbar_init_fence();
+
+  const uint64_t G = gridDim.x;
+  const uint64_t u0 = a.units * blockIdx.x / G;
+  const uint64_t u1 = a.units * (blockIdx.x + 1) / G;
+  const int64_t K = (int64_t)(u1 - u0);
+
+  auto unit_bytes = [&](uint64_t u, uint64_t &src_idx, uint64_t &off) -> uint32_t {
+    src_idx = u / a.tiles_per_src;
+    off = (u - src_idx * a.tiles_per_src) * kTile;
+    const uint64_t rem = a.src_bytes - off;
+    return (uint32_t)(rem < kTile ? rem : kTile);
+  };
+
+  bool failed = false;
+  int64_t loads_issued = 0, loads_seen = 0;
+  for (int64_t k = 0; k < K + kLookahead && !failed; ++k) {
+    if (k < K) {  // refill stage k % S with unit u0 + k
+      const int s = (int)(k % kStages);
+      if (k >= kStages) bulk_wait_read<kStages - kLookahead - 1>();
+      uint64_t r, off;
+      const uint32_t bytes = unit_bytes(u0 + k, r, off);
+      mbar_arrive_expect_tx(&bars[s], bytes);
+      bulk_load(smem + (size_t)s * kTile, a.src[r] + off, bytes, &bars[s]);
+      ++loads_issued;
+    }
+    const int64_t j = k - kLookahead;
+    if (j >= 0 && j < K) {  // write unit u0 + j to every destination
+      const int s = (int)(j % kStages);
+      if (!mbar_wait_bounded(&bars[s], (uint32_t)((j / kStages) & 1), kWaitLimitNs)) {
+        failed = true;
+        break;
+      }
+      ++loads_seen;
+      fence_proxy_async_smem();
+      uint64_t r, off;
+      const uint32_t bytes = unit_bytes(u0 + j, r, off);
+      const unsigned char *tile = smem + (size_t)s * kTile;
+      for (int q = 0; q < a.p; ++q) {
+        if ((a.skip[q] >> r) & 1u) continue;
+        bulk_store(a.dst[q] + r * a.src_bytes + off, tile, bytes);
+      }
+      bulk_commit();
+    }
+  }
+  if (failed) {
+    atomicAdd(&g_wait_timeouts, 1u);
+    // drain loads still in flight into this CTA's shared memory (bounded)
+    for (int64_t j = loads_seen; j < loads_issued; ++j) {
+      const int s = (int)(j % kStages);
+      if (!mbar_wait_bounded(&bars[s], (uint32_t)((j / kStages) & 1), kWaitLimitNs)) break;
+    }
+  }
+  bulk_wait_all();
+}
+
+// Fallback for buffers that are not 16-byte aligned (or sizes not a multiple
+// of 16 bytes): element copies, blockIdx.y = destination rank, x grid-stride.
+template <typename E>
+__global__ void fanout_elem_kernel(const __grid_constant__ FanoutParams a, int nsrc) {
+  const int q = blockIdx.y;
+  const uint64_t per_src = a.src_bytes / sizeof(E);
+  const uint64_t total = per_src * nsrc;
+  E *out = reinterpret_cast<E *>(a.dst[q]);
+  for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < total;
+       i += (uint64_t)gridDim.x * blockDim.x) {
+    const uint64_t r = i / per_src;
+    if ((a.skip[q] >> r) & 1u) continue;
+    out[i] = reinterpret_cast<const E *>(a.src[r])[i - r * per_src];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s) {
+  FanoutParams a{};
+  a.p = job.p;
+  a.src_bytes = job.src_bytes;
+  bool aligned = (job.src_bytes % 16 == 0);
+  for (int r = 0; r < job.nsrc; ++r) {
+    a.src[r] = static_cast<const char *>(job.src[r]);
+    aligned = aligned && reinterpret_cast<uintptr_t>(job.src[r]) % 16 == 0;
+  }
+  for (int q = 0; q < job.p; ++q) {
+    a.dst[q] = static_cast<char *>(job.dst[q]);
+    a.skip[q] = job.skip[q];
+    aligned = aligned && reinterpret_cast<uintptr_t>(job.dst[q]) % 16 == 0;
+  }
+  if (job.src_bytes == 0) return cudaSuccess;
+  cudaError_t err;
+  const int sms = device_sm_count();
+  if (aligned) {
+    a.tiles_per_src = (job.src_bytes + kTile - 1) / kTile;
+    a.units = a.tiles_per_src * job.nsrc;
+    const size_t smem = (size_t)kStages * kTile;
+    static std::atomic<uint64_t> attr_set{0};  // one bit per device
+    int dev = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_set.load() & bit)) {
+      err = cudaFuncSetAttribute(fanout_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+      if (err != cudaSuccess) return err;
+      attr_set.fetch_or(bit);
+    }
+    const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(sms, a.units));
+    fanout_bulk_kernel<<<(unsigned)grid, 32, smem, s>>>(a);
+  } else {
+    const uint64_t per_src = job.src_bytes / job.elem_bytes;
+    const uint64_t total = per_src * job.nsrc;
+    const unsigned gx = (unsigned)std::max<uint64_t>(
+        1, std::min<uint64_t>((total + 255) / 256, (uint64_t)sms * 4));
+    dim3 grid(gx, job.p);
+    if (job.elem_bytes == 2) fanout_elem_kernel<uint16_t><<<grid, 256, 0, s>>>(a, job.nsrc);
+    else fanout_elem_kernel<uint32_t><<<grid, 256, 0, s>>>(a, job.nsrc);
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_wait_timeouts(unsigned int *count) {
+  unsigned int zero = 0;
+  cudaError_t err = cudaMemcpyFromSymbol(count, g_wait_timeouts, sizeof(unsigned int));
+  if (err != cudaSuccess) return err;
+  if (*count) err = cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(unsigned int));
+  return err;
+}
+
+}  // namespace rc

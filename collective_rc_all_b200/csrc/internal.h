@@ -1,0 +1,76 @@
+// internal.h -- job descriptions passed from the C ABI layer (api.cu) to the
+// kernel launchers.  Not part of the public interface.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace rc {
+
+constexpr int kMaxP = 16;
+
+// Where a flat reduction writes its result.
+enum ReduceMode : int {
+  kModeAll = 0,      // every rank's recv buffer (all-reduce)
+  kModeOne = 1,      // one buffer (reduce to root)
+  kModeScatter = 2,  // chunk c to rank c's buffer at offset i - c*C (reduce-scatter)
+};
+
+struct ReduceJob {
+  const void *src[kMaxP];
+  void *dst[kMaxP];  // kModeAll: p buffers; kModeOne: dst[0]; kModeScatter: p shard buffers
+  int p;
+  uint64_t n;  // per-rank full-vector length
+  int in_dt, out_dt, op;
+  float scale;
+  int mode;
+  int ndst;  // kModeAll: number of outputs (0 means p)
+};
+
+struct FanoutJob {
+  const void *src[kMaxP];  // nsrc sources of src_bytes each
+  void *dst[kMaxP];        // p destinations; source r lands at dst[q] + r * src_bytes
+  int nsrc;                // p (all-gather) or 1 (broadcast)
+  int p;
+  uint64_t src_bytes;
+  uint32_t elem_bytes;     // 2 or 4 (for the unaligned fallback)
+  uint32_t skip[kMaxP];    // bit r of skip[q]: leave (source r -> rank q) alone (in place)
+};
+
+struct RingJob {
+  const void *x[kMaxP];  // send
+  void *y[kMaxP];        // recv
+  void *ws;              // fp32 partials when dt is bf16: 2 * p * C floats
+  int p;
+  uint64_t n;
+  int dt, op;
+  float scale;
+};
+
+struct HierJob {
+  const void *x[kMaxP];
+  void *y[kMaxP];
+  void *ws;  // staged variant: (ng + 1) * n accumulator values
+  int p, G;
+  uint64_t n;
+  int dt, op;
+  float scale;
+};
+
+cudaError_t launch_reduce(const ReduceJob &job, cudaStream_t s);
+cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s);
+cudaError_t launch_ring_literal(const RingJob &job, cudaStream_t s);
+cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s);
+cudaError_t launch_hier_staged(const HierJob &job, cudaStream_t s);
+cudaError_t launch_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);
+
+// Device-side bounded waits report here (fanout.cu).
+cudaError_t read_and_clear_wait_timeouts(unsigned int *count);
+
+// Helpers shared by the launchers (api.cu).
+int device_sm_count();        // SMs of the current device (cached)
+void note_launches(int k);    // count kernels launched
+int env_int(const char *name, int dflt);
+
+}  // namespace rc

@@ -1,0 +1,259 @@
+// reduce.cu -- the flat p-source reduction: one-shot all-reduce, reduce to
+// root, and reduce-scatter (fused with the scale and the output cast).
+//
+// Pages: "分布式训练/推理", section "通信原语：rank、world size 和 collective
+// operations" (y = sum_r x_r, reduce-scatter keeps one slice of it), section
+// "FSDP 的执行顺序" ((1/N_d) sum of gradients, reduce-scattered), and
+// "LLM Parallelism 基础", section "Ring AllReduce" for the fold order.
+//
+// Design (HBM-bound: (p-1) adds per element, 0.1 flop/byte at p = 8):
+//  * One thread owns whole 16-byte vectors: it issues all p 128-bit loads of
+//    ILP vectors before folding, so each thread keeps p*ILP*16 bytes in
+//    flight (256 B at p = 8) with no shared memory and no barriers.
+//  * The fold order of element i depends only on its chunk c = i / C:
+//    ranks (c+1)%p, ..., c.  Vectors never straddle a chunk (C % VEC == 0 is
+//    required for the vector path), so the rotated rank list is computed once
+//    per chunk segment and the p loads land in statically indexed registers.
+//  * Grid = (SMs x resident CTAs); CTA b owns the contiguous vector range
+//    [b*NV/G, (b+1)*NV/G): every CTA gets the same work to within one vector,
+//    so there is no partial last wave.
+//  * Results are written once per destination with 16-byte stores (8-byte for
+//    an fp32 -> bf16 reduce-scatter).
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace rc {
+namespace {
+
+constexpr int kNT = 256;
+
+struct ReduceParams {
+  const char *src[kMaxRanks];
+  char *dst[kMaxRanks];  // kModeScatter: dst[c] already offset by -c*C elements
+  uint64_t n;            // elements per rank
+  uint64_t C;            // chunk length ceil(n/p)
+  uint64_t nvec;         // number of units the grid splits (vectors or elements)
+  float scale;
+  int p;
+  int mode;
+  int ndst;  // outputs in kModeAll
+};
+
+template <int PMAX>
+constexpr int ilp_for() {
+  return PMAX <= 4 ? 4 : (PMAX <= 8 ? 2 : 1);
+}
+
+__device__ __forceinline__ int rot(uint64_t c, int k, int p) {
+  int r = (int)c + 1 + k;  // c < p, k < p  ->  r < 2p
+  return r >= p ? r - p : r;
+}
+
+template <int PMAX, class TI, class TO, int OP, bool VECTOR>
+__global__ void __launch_bounds__(kNT) reduce_kernel(const __grid_constant__ ReduceParams a) {
+  using Acc = typename TI::Acc;
+  constexpr int VEC = VECTOR ? kVec<TI> : 1;
+  constexpr int ILP = VECTOR ? ilp_for<PMAX>() : 1;
+  const int p = a.p;
+  const int tid = threadIdx.x;
+
+  // This CTA's share of the unit range (units = vectors, or elements).
+  const uint64_t G = gridDim.x;
+  uint64_t u0 = a.nvec * blockIdx.x / G;
+  const uint64_t u1 = a.nvec * (blockIdx.x + 1) / G;
+
+  while (u0 < u1) {
+    // chunk segment: all units in [u0, useg) share chunk c
+    const uint64_t c = (u0 * VEC) / a.C;
+    const uint64_t chunk_end_unit = ((c + 1) * a.C) / VEC;
+    const uint64_t useg = u1 < chunk_end_unit ? u1 : chunk_end_unit;
+
+    const char *s[PMAX];
+#pragma unroll
+    for (int k = 0; k < PMAX; ++k) s[k] = (k < p) ? a.src[rot(c, k, p)] : nullptr;
+    char *dscatter = a.dst[a.mode == kModeScatter ? c : 0];
+
+    for (uint64_t u = u0 + tid; u < useg; u += (uint64_t)kNT * ILP) {
+      uint4 raw[ILP][PMAX];
+      Acc sv[ILP][PMAX];
+      bool live[ILP];
+#pragma unroll
+      for (int j = 0; j < ILP; ++j) {
+        const uint64_t uj = u + (uint64_t)j * kNT;
+        live[j] = uj < useg;
+        if (live[j]) {
+#pragma unroll
+          for (int k = 0; k < PMAX; ++k) {
+            if (k < p) {
+              if constexpr (VECTOR) {
+                raw[j][k] = ld_stream_v4(s[k] + uj * 16);
+              } else {
+                sv[j][k] = load_elem<TI>(s[k], uj);
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < ILP; ++j) {
+        if (!live[j]) continue;
+        const uint64_t e = (u + (uint64_t)j * kNT) * VEC;  // first element
+        Acc acc[VEC];
+        if constexpr (VECTOR) {
+          unpack<TI>(raw[j][0], acc);
+#pragma unroll
+          for (int k = 1; k < PMAX; ++k) {
+            if (k < p) {
+              Acc v[VEC];
+              unpack<TI>(raw[j][k], v);
+#pragma unroll
+              for (int q = 0; q < VEC; ++q) acc[q] = combine<OP>(acc[q], v[q]);
+            }
+          }
+        } else {
+          acc[0] = sv[j][0];
+#pragma unroll
+          for (int k = 1; k < PMAX; ++k)
+            if (k < p) acc[0] = combine<OP>(acc[0], sv[j][k]);
+        }
+#pragma unroll
+        for (int q = 0; q < VEC; ++q) acc[q] = finish<OP>(acc[q], a.scale);
+
+        if (a.mode == kModeAll) {
+#pragma unroll
+          for (int r = 0; r < PMAX; ++r) {
+            if (r < a.ndst) {
+              if constexpr (VECTOR) store_vec<TO, VEC>(a.dst[r] + e * TO::kBytes, acc);
+              else store_elem<TO>(a.dst[r], e, acc[0]);
+            }
+          }
+        } else {
+          char *d = (a.mode == kModeScatter) ? dscatter : a.dst[0];
+          if constexpr (VECTOR) store_vec<TO, VEC>(d + e * TO::kBytes, acc);
+          else store_elem<TO>(d, e, acc[0]);
+        }
+      }
+    }
+    u0 = useg;
+  }
+}
+
+// Elements past the last whole vector (n % VEC of them, all in the last
+// chunk) -- one small CTA, scalar.
+template <int PMAX, class TI, class TO, int OP>
+__global__ void __launch_bounds__(32) reduce_tail_kernel(const __grid_constant__ ReduceParams a,
+                                                          uint64_t first) {
+  using Acc = typename TI::Acc;
+  const int p = a.p;
+  for (uint64_t e = first + threadIdx.x; e < a.n; e += blockDim.x) {
+    const uint64_t c = e / a.C;
+    Acc acc = load_elem<TI>(a.src[rot(c, 0, p)], e);
+    for (int k = 1; k < p; ++k) acc = combine<OP>(acc, load_elem<TI>(a.src[rot(c, k, p)], e));
+    acc = finish<OP>(acc, a.scale);
+    if (a.mode == kModeAll) {
+      for (int r = 0; r < a.ndst; ++r) store_elem<TO>(a.dst[r], e, acc);
+    } else {
+      store_elem<TO>(a.dst[a.mode == kModeScatter ? c : 0], e, acc);
+    }
+  }
+}
+
+template <int PMAX, class TI, class TO, int OP>
+cudaError_t run(const ReduceJob &job, cudaStream_t s) {
+  ReduceParams a{};
+  const int p = job.p;
+  const uint64_t n = job.n;
+  const uint64_t C = (n + p - 1) / p;
+  a.n = n;
+  a.C = C;
+  a.p = p;
+  a.mode = job.mode;
+  a.scale = job.scale;
+  a.ndst = job.mode == kModeAll ? (job.ndst > 0 ? job.ndst : p) : 1;
+  bool aligned = true;
+  for (int r = 0; r < p; ++r) {
+    a.src[r] = static_cast<const char *>(job.src[r]);
+    aligned = aligned && (reinterpret_cast<uintptr_t>(job.src[r]) % 16 == 0);
+  }
+  const int ndst = job.mode == kModeOne ? 1 : (job.mode == kModeAll ? a.ndst : p);
+  for (int r = 0; r < ndst; ++r) {
+    uintptr_t d = reinterpret_cast<uintptr_t>(job.dst[r]);
+    aligned = aligned && (d % 16 == 0);
+    if (job.mode == kModeScatter) d -= (uintptr_t)(r * C * TO::kBytes);  // index by global element
+    a.dst[r] = reinterpret_cast<char *>(d);
+  }
+  constexpr int VEC = kVec<TI>;
+  const bool vector = aligned && (C % VEC == 0);
+
+  const int sms = device_sm_count();
+  cudaError_t err;
+  if (vector) {
+    auto kern = reduce_kernel<PMAX, TI, TO, OP, true>;
+    int occ = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNT, 0);
+    if (err != cudaSuccess) return err;
+    occ = std::max(1, std::min(occ, env_int("RC_CTAS_PER_SM", occ)));
+    a.nvec = n / VEC;
+    if (a.nvec > 0) {
+      const uint64_t per_cta_min = (uint64_t)kNT;  // at least one vector per thread
+      uint64_t grid = std::min<uint64_t>((uint64_t)sms * occ, (a.nvec + per_cta_min - 1) / per_cta_min);
+      grid = std::max<uint64_t>(grid, 1);
+      kern<<<(unsigned)grid, kNT, 0, s>>>(a);
+      note_launches(1);
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    if (a.nvec * VEC < n) {
+      reduce_tail_kernel<PMAX, TI, TO, OP><<<1, 32, 0, s>>>(a, a.nvec * VEC);
+      note_launches(1);
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+  } else {
+    auto kern = reduce_kernel<PMAX, TI, TO, OP, false>;
+    int occ = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNT, 0);
+    if (err != cudaSuccess) return err;
+    a.nvec = n;
+    uint64_t grid = std::min<uint64_t>((uint64_t)sms * std::max(occ, 1), (n + kNT - 1) / kNT);
+    grid = std::max<uint64_t>(grid, 1);
+    kern<<<(unsigned)grid, kNT, 0, s>>>(a);
+    note_launches(1);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+template <class TI, class TO, int OP>
+cudaError_t by_p(const ReduceJob &job, cudaStream_t s) {
+  // PMAX bounds both the sources and (for kModeAll) the outputs
+  const int w = std::max(job.p, job.mode == kModeAll && job.ndst > 0 ? job.ndst : job.p);
+  if (w <= 2) return run<2, TI, TO, OP>(job, s);
+  if (w <= 4) return run<4, TI, TO, OP>(job, s);
+  if (w <= 8) return run<8, TI, TO, OP>(job, s);
+  return run<16, TI, TO, OP>(job, s);
+}
+
+template <class TI, class TO>
+cudaError_t by_op(const ReduceJob &job, cudaStream_t s) {
+  switch (job.op) {
+    case kSum: return by_p<TI, TO, kSum>(job, s);
+    case kMax: return by_p<TI, TO, kMax>(job, s);
+    case kMin: return by_p<TI, TO, kMin>(job, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_reduce(const ReduceJob &job, cudaStream_t s) {
+  const int i = job.in_dt, o = job.out_dt;
+  if (i == kF32 && o == kF32) return by_op<F32, F32>(job, s);
+  if (i == kBF16 && o == kBF16) return by_op<BF16, BF16>(job, s);
+  if (i == kI32 && o == kI32) return by_op<I32, I32>(job, s);
+  if (i == kF32 && o == kBF16) return by_op<F32, BF16>(job, s);
+  if (i == kBF16 && o == kF32) return by_op<BF16, F32>(job, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rc

@@ -1,0 +1,296 @@
+// ring.cu -- the literal ring all-reduce, executed step by step.
+//
+// Page: "LLM Parallelism 基础", section "Ring AllReduce": the data is cut into
+// N chunks; in the reduce-scatter phase (N-1 steps) every card sends one
+// chunk to the next card on the ring, which accumulates it into its own
+// matching chunk, so that card 0 ends up with the finished chunk 0; in the
+// all-gather phase (N-1 steps) every card forwards its finished chunk to the
+// next card, which overwrites its copy.  2(N-1) steps in all.  The bandwidth
+// model is in "分布式训练/推理", section "Ring all-reduce 的带宽账".
+//
+// Schedule executed here, for p simulated ranks held in one GPU's memory:
+//   reduce-scatter step k = 0..p-2, every rank r:
+//     c = (r-k-1) mod p, d = r+1 mod p
+//     msg = (k == 0) ? x_r[chunk c] : partial_r[chunk c]       (the send)
+//     partial_d[chunk c] = msg (+) x_d[chunk c]                (the receive)
+//     at k = p-2 the receiver owns chunk c == d: y_d[chunk d] = cast(scale*acc)
+//   all-gather step k = 0..p-2, every rank r:
+//     c = (r-k) mod p:  y_{r+1}[chunk c] = y_r[chunk c]
+// Every send and receive is a real load / store in device memory.  Partials
+// are fp32 (int32 for int32): they live in the receiver's own y buffer for
+// fp32/int32 and in a workspace [2 parities][p][C] for bf16 (the parity
+// double-buffers consecutive steps).
+//
+// Tile-outer / step-inner: each thread owns fixed offsets o inside the
+// chunks and runs all 2(p-1) steps on them.  Step k+1 reads exactly what
+// the same thread stored at step k, so program order is the only
+// synchronisation -- no grid barrier, no flags, nothing can wait forever.
+// Within one step the ranks' reads and writes touch disjoint locations, so a
+// thread issues the loads of a group of RG ranks before any of their stores
+// (memory-level parallelism) without changing the schedule's result.
+#include <algorithm>
+#include <type_traits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace rc {
+namespace {
+
+constexpr int kRingNT = 128;
+
+struct RingParams {
+  const char *x[kMaxRanks];
+  char *y[kMaxRanks];
+  char *ws;
+  uint64_t n, C;
+  uint64_t units;  // units (vectors or elements) per chunk
+  float scale;
+  int p;
+};
+
+// Coherent loads at L2 (partials are written and read back in this kernel).
+__device__ __forceinline__ uint4 ld_cg_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_cg_u32(const void *p) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_cg_u16(const void *p) {
+  unsigned short v;
+  asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_u32(void *p, uint32_t v) {
+  asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_u16(void *p, uint32_t v) {
+  asm volatile("st.global.u16 [%0], %1;" ::"l"(p), "h"((unsigned short)v) : "memory");
+}
+
+// input element(s) of type T -> accumulators
+template <class T, int VEC>
+__device__ __forceinline__ void load_in(const char *p, typename T::Acc (&a)[VEC]) {
+  if constexpr (VEC == 1) {
+    if constexpr (std::is_same<T, BF16>::value) a[0] = bf16_bits_to_f32(ld_cg_u16(p));
+    else if constexpr (std::is_same<T, F32>::value) a[0] = __uint_as_float(ld_cg_u32(p));
+    else a[0] = (int32_t)ld_cg_u32(p);
+  } else {
+    unpack<T>(ld_cg_v4(p), a);
+  }
+}
+
+// partial (raw 32-bit accumulators) load / store
+template <class Acc, int VEC>
+__device__ __forceinline__ void load_part(const char *p, Acc (&a)[VEC]) {
+  uint32_t w[VEC];
+  if constexpr (VEC == 1) {
+    w[0] = ld_cg_u32(p);
+  } else {
+#pragma unroll
+    for (int h = 0; h < VEC / 4; ++h) {
+      const uint4 v = ld_cg_v4(p + 16 * h);
+      w[4 * h] = v.x;
+      w[4 * h + 1] = v.y;
+      w[4 * h + 2] = v.z;
+      w[4 * h + 3] = v.w;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) {
+    if constexpr (std::is_same<Acc, float>::value) a[j] = __uint_as_float(w[j]);
+    else a[j] = (int32_t)w[j];
+  }
+}
+__device__ __forceinline__ uint32_t acc_bits(float v) { return __float_as_uint(v); }
+__device__ __forceinline__ uint32_t acc_bits(int32_t v) { return (uint32_t)v; }
+
+template <class Acc, int VEC>
+__device__ __forceinline__ void store_part(char *p, const Acc (&a)[VEC]) {
+  if constexpr (VEC == 1) {
+    st_u32(p, acc_bits(a[0]));
+  } else {
+#pragma unroll
+    for (int h = 0; h < VEC / 4; ++h)
+      st_v4(p + 16 * h, make_uint4(acc_bits(a[4 * h]), acc_bits(a[4 * h + 1]),
+                                   acc_bits(a[4 * h + 2]), acc_bits(a[4 * h + 3])));
+  }
+}
+
+template <class T, int VEC>
+__device__ __forceinline__ void store_out(char *p, const typename T::Acc (&a)[VEC]) {
+  if constexpr (VEC == 1) {
+    if constexpr (std::is_same<T, BF16>::value) st_u16(p, f32_to_bf16_bits(a[0]));
+    else st_u32(p, acc_bits(a[0]));
+  } else {
+    store_vec<T, VEC>(p, a);
+  }
+}
+
+__device__ __forceinline__ int mod_p(int v, int p) { return v < 0 ? v + p : v; }
+
+template <class T, int OP, bool VECTOR, int RG>
+__global__ void __launch_bounds__(kRingNT) ring_literal_kernel(const __grid_constant__ RingParams a) {
+  using Acc = typename T::Acc;
+  constexpr int VEC = VECTOR ? kVec<T> : 1;
+  constexpr bool kWs = std::is_same<T, BF16>::value;  // bf16: fp32 partials in workspace
+  const int p = a.p;
+  const uint64_t C = a.C;
+
+  auto chunk_len = [&](int c) -> uint64_t {
+    const uint64_t b = (uint64_t)c * C;
+    return b >= a.n ? 0 : (a.n - b < C ? a.n - b : C);
+  };
+  // where rank `rank` keeps its partial of chunk c for step parity `par`
+  auto part = [&](int rank, int c, int par, uint64_t oe) -> char * {
+    if constexpr (kWs) return a.ws + (((uint64_t)(par * p + rank)) * C + oe) * 4;
+    else return a.y[rank] + ((uint64_t)c * C + oe) * 4;
+  };
+
+  const uint64_t G = gridDim.x;
+  const uint64_t o0 = a.units * blockIdx.x / G;
+  const uint64_t o1 = a.units * (blockIdx.x + 1) / G;
+
+  for (uint64_t o = o0 + threadIdx.x; o < o1; o += blockDim.x) {
+    const uint64_t oe = o * VEC;  // element offset inside every chunk
+
+    // ---- phase 1: reduce-scatter, p-1 steps
+    for (int k = 0; k + 1 < p; ++k) {
+      const bool last = (k + 2 == p);
+      for (int r0 = 0; r0 < p; r0 += RG) {
+        Acc msg[RG][VEC], own[RG][VEC];
+        bool act[RG];
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {  // all sends/receives' loads first
+          const int r = r0 + g;
+          act[g] = false;
+          if (r < p) {
+            const int c = mod_p(r - k - 1, p);
+            const int d = (r + 1 < p) ? r + 1 : 0;
+            if (oe < chunk_len(c)) {
+              act[g] = true;
+              const uint64_t e = (uint64_t)c * C + oe;
+              if (k == 0) load_in<T, VEC>(a.x[r] + e * T::kBytes, msg[g]);
+              else load_part<Acc, VEC>(part(r, c, (k - 1) & 1, oe), msg[g]);
+              load_in<T, VEC>(a.x[d] + e * T::kBytes, own[g]);
+            }
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {  // then the folds and stores
+          if (!act[g]) continue;
+          const int r = r0 + g;
+          const int c = mod_p(r - k - 1, p);
+          const int d = (r + 1 < p) ? r + 1 : 0;
+#pragma unroll
+          for (int j = 0; j < VEC; ++j) msg[g][j] = combine<OP>(msg[g][j], own[g][j]);
+          if (last) {  // receiver d now owns the finished chunk c (== d)
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) msg[g][j] = finish<OP>(msg[g][j], a.scale);
+            store_out<T, VEC>(a.y[d] + ((uint64_t)c * C + oe) * T::kBytes, msg[g]);
+          } else {
+            store_part<Acc, VEC>(part(d, c, k & 1, oe), msg[g]);
+          }
+        }
+      }
+    }
+
+    // ---- phase 2: all-gather, p-1 steps, the receiver overwrites
+    for (int k = 0; k + 1 < p; ++k) {
+      for (int r0 = 0; r0 < p; r0 += RG) {
+        uint4 v16[RG];
+        uint32_t v4[RG];
+        bool act[RG];
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {
+          const int r = r0 + g;
+          act[g] = false;
+          if (r < p) {
+            const int c = mod_p(r - k, p);
+            if (oe < chunk_len(c)) {
+              act[g] = true;
+              const char *src = a.y[r] + ((uint64_t)c * C + oe) * T::kBytes;
+              if constexpr (VECTOR) v16[g] = ld_cg_v4(src);
+              else if constexpr (T::kBytes == 2) v4[g] = ld_cg_u16(src);
+              else v4[g] = ld_cg_u32(src);
+            }
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {
+          if (!act[g]) continue;
+          const int r = r0 + g;
+          const int c = mod_p(r - k, p);
+          const int d = (r + 1 < p) ? r + 1 : 0;
+          char *dst = a.y[d] + ((uint64_t)c * C + oe) * T::kBytes;
+          if constexpr (VECTOR) st_v4(dst, v16[g]);
+          else if constexpr (T::kBytes == 2) st_u16(dst, v4[g]);
+          else st_u32(dst, v4[g]);
+        }
+      }
+    }
+  }
+}
+
+template <class T, int OP>
+cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
+  RingParams a{};
+  const int p = job.p;
+  a.p = p;
+  a.n = job.n;
+  a.C = (job.n + p - 1) / p;
+  a.scale = job.scale;
+  a.ws = static_cast<char *>(job.ws);
+  bool aligned = reinterpret_cast<uintptr_t>(job.ws) % 16 == 0;
+  for (int r = 0; r < p; ++r) {
+    a.x[r] = static_cast<const char *>(job.x[r]);
+    a.y[r] = static_cast<char *>(job.y[r]);
+    aligned = aligned && reinterpret_cast<uintptr_t>(job.x[r]) % 16 == 0 &&
+              reinterpret_cast<uintptr_t>(job.y[r]) % 16 == 0;
+  }
+  constexpr int VEC = kVec<T>;
+  const bool vector = aligned && a.C % VEC == 0 && a.n % VEC == 0;
+  constexpr int RG = std::is_same<T, BF16>::value ? 4 : 8;
+  const int sms = device_sm_count();
+  auto kern = vector ? ring_literal_kernel<T, OP, true, RG> : ring_literal_kernel<T, OP, false, RG>;
+  a.units = vector ? a.C / VEC : a.C;
+  int occ = 0;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kRingNT, 0);
+  if (err != cudaSuccess) return err;
+  occ = std::max(1, std::min(occ, env_int("RC_CTAS_PER_SM", occ)));
+  uint64_t grid = std::min<uint64_t>((uint64_t)sms * occ, (a.units + kRingNT - 1) / kRingNT);
+  grid = std::max<uint64_t>(grid, 1);
+  kern<<<(unsigned)grid, kRingNT, 0, s>>>(a);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+template <class T>
+cudaError_t ring_by_op(const RingJob &job, cudaStream_t s) {
+  switch (job.op) {
+    case kSum: return run_ring<T, kSum>(job, s);
+    case kMax: return run_ring<T, kMax>(job, s);
+    case kMin: return run_ring<T, kMin>(job, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_ring_literal(const RingJob &job, cudaStream_t s) {
+  switch (job.dt) {
+    case kF32: return ring_by_op<F32>(job, s);
+    case kBF16: return ring_by_op<BF16>(job, s);
+    case kI32: return ring_by_op<I32>(job, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rc

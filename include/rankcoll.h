@@ -1,0 +1,212 @@
+/*
+ * rankcoll.h -- C ABI of librankcoll: collective reductions over p simulated
+ * ranks whose buffers all live in one GPU's memory (sm_100a, B200).
+ *
+ * Every rank is a separate device buffer.  A call takes host arrays of p
+ * device pointers (one per rank), a per-rank element count, a dtype, a
+ * reduction op, an fp32 scale and a CUDA stream.  All work runs in this
+ * library's own CUDA kernels, enqueued on the caller's stream.
+ *
+ * Sources, cited as page title and section:
+ *  [SEM]  "分布式训练/推理" (llm-from-scratch, chapter 7), section
+ *         "通信原语：rank、world size 和 collective operations" -- the primitive
+ *         table (broadcast, reduce with sum/min/max, all-gather, reduce-scatter,
+ *         all-reduce), y = sum_r x_r, the four-rank worked example, and
+ *         all_reduce = reduce_scatter + all_gather.
+ *  [API]  same page, "PyTorch distributed：代码里真正发生了什么" -- all_reduce
+ *         works in place; reduce_scatter takes a world_size x k input and a
+ *         separate k output; all_gather writes a separate full output.
+ *  [AVG]  same page, "数据并行：切 batch，复制模型" -- the gradient average
+ *         g = (1/p) sum_r grad L_r (ReduceOp.AVG), here `scale` = 1/p.
+ *  [FSDP] same page, "FSDP 的执行顺序：常驻 shard，计算前 gather，反向后 scatter" --
+ *         all_gather of parameter shards, reduce_scatter of (1/N_d) sum of grads.
+ *  [COLL] "LLM Parallelism 基础", sections "AllReduce" and "其他 Collective" --
+ *         Reduce (result on one process), Broadcast, AllGather, ReduceScatter.
+ *  [RING] same page, section "Ring AllReduce" -- N chunks; reduce-scatter phase
+ *         of N-1 steps (send one chunk to the next card, which accumulates);
+ *         all-gather phase of N-1 steps (forward the finished chunk, receiver
+ *         overwrites); 2(N-1) steps; card 0 ends the first phase holding chunk 0.
+ *  [HIER] "大模型并行的最小闭环：集合通信、TP、FSDP/ZeRO-3 到权重分片", log excerpt
+ *         "分层 AllReduce + SHARP", steps 1-6 -- intra-node AllReduce, one
+ *         representative per node, the node results added together, intra-node
+ *         broadcast.
+ *
+ * Result contract (identical bits on every call, checked against an
+ * independent CPU implementation):
+ *  - Chunk length C = ceil(n/p); element i lies in chunk c = i / C.  Every
+ *    reducing call folds the ranks of element i in the order the ring of
+ *    [RING] produces: x_{(c+1)%p}, then x_{(c+2)%p}, ..., last x_{c}, starting
+ *    from the first operand (no identity element).
+ *  - fp32 and bf16 inputs accumulate in fp32 (IEEE round-to-nearest-even,
+ *    no fused multiply-add, no flush to zero); `scale` is one fp32 multiply
+ *    after the fold; a bf16 output is one round-to-nearest-even at the end.
+ *  - int32 SUM wraps (two's complement).  MAX / MIN are compare-selects
+ *    (acc = v > acc ? v : acc), so a tie keeps the earlier operand.
+ *  - `scale` must be 1.0f unless op is RC_SUM on a floating type.
+ *
+ * Common argument rules:
+ *  - p in [1, 16].  n = per-rank length of the full vector (elements).
+ *    n == 0 returns RC_OK and launches nothing.
+ *  - Pointer arrays are host memory owned by the caller, read only during the
+ *    call (their contents are copied into kernel parameters).  Device buffers
+ *    belong to the caller and must stay valid until the stream work is done.
+ *  - Aliasing: output buffers must not overlap each other.  An output may
+ *    overlap an input only when both describe the same elements at the same
+ *    addresses (e.g. in-place all_reduce recv[r] == send[r], or a
+ *    reduce_scatter output recv[r] == send[r] + r*(n/p) with equal element
+ *    sizes).  Any other overlap returns RC_ERR_INVALID_ARG.
+ *  - Pointers need no particular alignment; 16-byte aligned buffers (and
+ *    chunk lengths that keep 16-byte alignment) take the vectorised path.
+ *  - Calls are asynchronous and stream-ordered.  Argument errors are reported
+ *    before anything is enqueued.  A failed launch returns RC_ERR_CUDA.
+ *    Faults that happen later on the device surface through rc_stream_status.
+ *  - Thread safety: calls may come from several host threads.  Calls that
+ *    use the library workspace (see each function) share it per (device,
+ *    stream), so calls on one stream are safe; the workspace of a stream is
+ *    grown in stream order.
+ */
+#ifndef RANKCOLL_H
+#define RANKCOLL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RC_OK = 0,
+    RC_ERR_INVALID_ARG = 1, /* bad pointer, size, dtype/op combination, alias */
+    RC_ERR_UNSUPPORTED = 2, /* valid request this build does not implement    */
+    RC_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed           */
+    RC_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up             */
+} rc_status;
+
+typedef enum { RC_FP32 = 0, RC_BF16 = 1, RC_INT32 = 2 } rc_dtype;
+typedef enum { RC_SUM = 0, RC_MAX = 1, RC_MIN = 2 } rc_op;
+typedef enum { RC_RING_LITERAL = 0, RC_RING_ONESHOT = 1 } rc_ring_variant;
+typedef enum { RC_HIER_FUSED = 0, RC_HIER_STAGED = 1 } rc_hier_variant;
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *rc_stream_t;
+
+/*
+ * all-reduce [SEM] [COLL] [AVG]: recv[r][i] = cast(scale * fold_r send[r][i])
+ * for every rank r.  send, recv: p device pointers to n elements of dt.
+ * One kernel launch: each element is read once per rank and written once per
+ * rank.  In place (recv[r] == send[r]) is allowed.
+ */
+rc_status rc_all_reduce(const void *const *send, void *const *recv, int p, size_t n,
+                        rc_dtype dt, rc_op op, float scale, rc_stream_t stream);
+
+/*
+ * reduce-scatter [SEM] [API] [FSDP]: rank r receives elements [r*m, (r+1)*m)
+ * of the all-reduce result, m = n/p, cast to out_dt.  send: p pointers to n
+ * elements of in_dt; recv: p pointers to m elements of out_dt.  n % p != 0
+ * is RC_ERR_INVALID_ARG.  (in_dt, out_dt) may be equal, or fp32->bf16 (the
+ * fused gradient path: scale 1/p and the bf16 cast in the same kernel), or
+ * bf16->fp32.  int32 only to int32.
+ */
+rc_status rc_reduce_scatter(const void *const *send, void *const *recv, int p, size_t n,
+                            rc_dtype in_dt, rc_dtype out_dt, rc_op op, float scale,
+                            rc_stream_t stream);
+
+/*
+ * all-gather [SEM] [API] [FSDP]: recv[q][r*m + j] = send[r][j] for every q;
+ * m = n/p.  send: p pointers to m elements; recv: p pointers to n elements.
+ * A byte copy (any dt).  If recv[q] + r*m*size == send[r] that slot is left
+ * as is.  Aligned data moves by bulk copies global -> shared -> global.
+ */
+rc_status rc_all_gather(const void *const *send, void *const *recv, int p, size_t n,
+                        rc_dtype dt, rc_stream_t stream);
+
+/*
+ * reduce [SEM] [COLL]: only the root receives the all-reduce result:
+ * recv_root[i] = cast(scale * fold_r send[r][i]).  root in [0, p) names the
+ * receiving rank (the fold order does not depend on it); recv_root may be
+ * send[root] (in place).
+ */
+rc_status rc_reduce(const void *const *send, void *recv_root, int p, int root, size_t n,
+                    rc_dtype dt, rc_op op, float scale, rc_stream_t stream);
+
+/*
+ * broadcast [SEM] [COLL]: recv[q][i] = send_root[i] for every q.  root in
+ * [0, p); if recv[root] == send_root the root's copy is skipped.
+ */
+rc_status rc_broadcast(const void *send_root, void *const *recv, int p, int root, size_t n,
+                       rc_dtype dt, rc_stream_t stream);
+
+/*
+ * ring all-reduce [RING]: same result bits as rc_all_reduce.
+ *  RC_RING_LITERAL executes the 2(p-1) steps: reduce-scatter step k, every
+ *   rank r sends chunk (r-k-1) mod p to rank r+1, which folds it with its own
+ *   chunk; all-gather step k, rank r forwards chunk (r-k) mod p to rank r+1,
+ *   which overwrites.  Partials are fp32 (int32 for int32): kept in the
+ *   receivers' recv buffers when dt is fp32/int32, in the library workspace
+ *   (2 * p * C * 4 bytes) when dt is bf16.  One persistent launch; each thread
+ *   block runs all steps on one offset range of every chunk.
+ *  RC_RING_ONESHOT reads all p ranks directly (the rc_all_reduce kernel).
+ */
+rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, size_t n,
+                             rc_dtype dt, rc_op op, float scale, rc_ring_variant variant,
+                             rc_stream_t stream);
+
+/*
+ * hierarchical all-reduce [HIER]: ranks form p/group_size contiguous groups
+ * of group_size.  (1) each group's ranks are folded in ring order over the
+ * group (chunk length ceil(n/group_size)); (2) the groups' results are folded
+ * in ring order over the groups (chunk length ceil(n/(p/group_size))); (3)
+ * scale and cast once, and every rank receives the result.  group_size must
+ * divide p.  Result bits differ from rc_all_reduce by rounding only (equal
+ * for int32, MAX, MIN).
+ *  RC_HIER_FUSED: one launch, group results in registers.
+ *  RC_HIER_STAGED: three launches (intra-group reduce to fp32 workspace,
+ *   leader sum, broadcast); workspace (p/group_size + 1) * n * 4 bytes.
+ */
+rc_status rc_hier_all_reduce(const void *const *send, void *const *recv, int p, int group_size,
+                             size_t n, rc_dtype dt, rc_op op, float scale,
+                             rc_hier_variant variant, rc_stream_t stream);
+
+/*
+ * Plain device copy dst[0, bytes) = src[0, bytes) with this library's
+ * streaming kernel: the measured copy roofline the collectives are judged
+ * against.  src and dst must not overlap.
+ */
+rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream);
+
+/* Validate a device range without launching anything: RC_OK when
+ * [ptr, ptr + bytes) is device (or managed) memory of the current device
+ * inside a single allocation, RC_ERR_INVALID_ARG otherwise (message in
+ * rc_last_error).  Every collective runs this check on each buffer. */
+rc_status rc_check_buffer(const void *ptr, size_t bytes);
+
+/* Grow the workspace of (current device, stream) to at least `bytes` now, so
+ * that later calls do not allocate.  Stream-ordered. */
+rc_status rc_reserve_workspace(size_t bytes, rc_stream_t stream);
+
+/* Synchronise `stream`, then report: RC_ERR_CUDA for an asynchronous CUDA
+ * error, RC_ERR_TIMEOUT if a bounded device wait of this library gave up
+ * since the last call (the flag is cleared), else RC_OK. */
+rc_status rc_stream_status(rc_stream_t stream);
+
+/* Static description of a status code. */
+const char *rc_status_string(rc_status status);
+
+/* Text of the last error raised on the calling host thread ("" if none). */
+const char *rc_last_error(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t rc_launch_count(void);
+
+/* Free every workspace (synchronises the devices that own one). */
+rc_status rc_finalize(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int rc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RANKCOLL_H */

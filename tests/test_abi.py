@@ -1,0 +1,94 @@
+"""The C ABI library loads and exports every entry point the header declares,
+and rejects bad arguments on the host before anything reaches a GPU.
+CPU only (no CUDA device needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "rankcoll.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rc_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def rc():
+    import collective_rc_all_b200 as m
+    return m
+
+
+def test_header_declares_the_collectives():
+    names = _declared()
+    for n in ("rc_all_reduce", "rc_reduce_scatter", "rc_all_gather", "rc_reduce", "rc_broadcast",
+              "rc_ring_all_reduce", "rc_hier_all_reduce"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(rc):
+    for name in _declared():
+        assert hasattr(rc.lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings(rc):
+    for code in range(5):
+        assert rc.lib.rc_status_string(code)
+    assert rc.rc_version() == 100
+
+
+def _null(p):
+    return (ctypes.c_void_p * p)(*([0] * p))
+
+
+def test_invalid_arguments_rejected_on_host(rc):
+    L = rc.lib
+    a = _null(16)
+    before = rc.rc_launch_count()
+    assert L.rc_all_reduce(a, a, 0, 10, 0, 0, 1.0, None) == 1          # p < 1
+    assert L.rc_all_reduce(a, a, 17, 10, 0, 0, 1.0, None) == 1         # p > 16
+    assert L.rc_all_reduce(a, a, 2, 10, 7, 0, 1.0, None) == 1          # dtype
+    assert L.rc_all_reduce(a, a, 2, 10, 0, 9, 1.0, None) == 1          # op
+    assert L.rc_all_reduce(a, a, 2, 10, 0, 1, 0.5, None) == 1          # scale with MAX
+    assert L.rc_all_reduce(a, a, 2, 10, 2, 0, 0.5, None) == 1          # scale with int32
+    assert L.rc_all_reduce(a, a, 2, 10, 0, 0, 1.0, None) == 1          # NULL buffers
+    assert "NULL" in rc.rc_last_error()
+    assert L.rc_reduce_scatter(a, a, 4, 10, 0, 0, 0, 1.0, None) == 1   # 4 does not divide 10
+    assert L.rc_reduce_scatter(a, a, 2, 10, 2, 0, 0, 1.0, None) == 1   # int32 -> fp32
+    assert L.rc_all_gather(a, a, 3, 10, 0, None) == 1                  # 3 does not divide 10
+    assert L.rc_reduce(a, None, 4, 4, 10, 0, 0, 1.0, None) == 1        # root out of range
+    assert L.rc_broadcast(None, a, 4, -1, 10, 0, None) == 1            # root out of range
+    assert L.rc_hier_all_reduce(a, a, 8, 3, 10, 0, 0, 1.0, 0, None) == 1   # 3 does not divide 8
+    assert L.rc_hier_all_reduce(a, a, 8, 4, 10, 0, 0, 1.0, 5, None) == 1   # variant
+    assert L.rc_ring_all_reduce(a, a, 8, 10, 0, 0, 1.0, 5, None) == 1      # variant
+    assert L.rc_all_reduce(None, None, 2, 10, 0, 0, 1.0, None) == 1    # NULL arrays
+    assert rc.rc_launch_count() == before
+
+
+def test_empty_calls_are_noops(rc):
+    L = rc.lib
+    a = _null(4)
+    before = rc.rc_launch_count()
+    assert L.rc_all_reduce(a, a, 4, 0, 0, 0, 1.0, None) == 0
+    assert L.rc_reduce_scatter(a, a, 4, 0, 0, 1, 0, 0.25, None) == 0
+    assert L.rc_all_gather(a, a, 4, 0, 1, None) == 0
+    assert L.rc_reduce(a, None, 4, 0, 0, 2, 1, 1.0, None) == 0
+    assert L.rc_broadcast(None, a, 4, 0, 0, 0, None) == 0
+    assert L.rc_ring_all_reduce(a, a, 4, 0, 0, 0, 1.0, 0, None) == 0
+    assert L.rc_hier_all_reduce(a, a, 4, 2, 0, 0, 0, 1.0, 1, None) == 0
+    assert rc.rc_launch_count() == before
+
+
+def test_host_memory_is_not_a_device_pointer(rc):
+    """Without a GPU (or with one) a host address is rejected, never launched."""
+    import numpy as np
+    x = [np.zeros(64, np.float32) for _ in range(2)]
+    ptr = (ctypes.c_void_p * 2)(*[v.ctypes.data for v in x])
+    before = rc.rc_launch_count()
+    assert rc.lib.rc_all_reduce(ptr, ptr, 2, 64, 0, 0, 1.0, None) == 1
+    assert rc.rc_launch_count() == before

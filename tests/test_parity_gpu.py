@@ -1,0 +1,444 @@
+"""GPU parity: every collective of the CUDA library against the CPU oracle on
+the same seeded inputs, compared bit for bit (the fold order, fp32
+accumulation and bf16 rounding are part of the contract, so "within
+tolerance" would hide a broken kernel).  Hierarchical vs flat all-reduce are
+two different orders and are compared with the fold bound
+|err| <= p * 2^-24 * sum_r |x_r| (plus one bf16 ulp for bf16 outputs).
+
+Sizes: small cases the oracle runs in full (several tiles, ragged tails),
+and the configs' full sizes -- compared in full where the oracle finishes in
+seconds, else on sampled indices (chunk boundaries included).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rc_inputs
+from util import assert_bits, check_canary, empty_dev, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+DTS = ["f32", "bf16", "i32"]
+OPS = ["sum", "max", "min"]
+ESZ = {"f32": 4, "bf16": 2, "i32": 4}
+
+
+@pytest.fixture(scope="module")
+def rc():
+    import collective_rc_all_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+def _data(p, n, dt, seed):
+    if dt == "i32":
+        return rc_inputs.int_uniform(p, n, seed)
+    return rc_inputs.uniform(p, n, seed, dt)
+
+
+def _sync(rc):
+    torch.cuda.synchronize()
+    rc.rc_stream_status()
+
+
+# ------------------------------------------------------------ worked example
+def test_worked_example(rc):
+    xs = rc_inputs.worked_example()
+    d, _ = to_dev(xs, "f32")
+    y, _ = empty_dev(4, "f32", 4)
+    rc.rc_all_reduce(d, y)
+    rs, _ = empty_dev(1, "f32", 4)
+    rc.rc_reduce_scatter(d, rs)
+    ag, _ = empty_dev(4, "f32", 4)
+    rc.rc_all_gather(rs, ag)
+    ring, _ = empty_dev(4, "f32", 4)
+    rc.rc_ring_all_reduce(d, ring)
+    _sync(rc)
+    for r in range(4):
+        assert to_host(y[r], "f32").tolist() == [6, 10, 14, 18]
+        assert to_host(rs[r], "f32").tolist() == [[6], [10], [14], [18]][r]
+        assert to_host(ag[r], "f32").tolist() == [6, 10, 14, 18]
+        assert to_host(ring[r], "f32").tolist() == [6, 10, 14, 18]
+
+
+def test_ring_order_golden(rc):
+    """Hand-derived ring-order case: the ring order gives 0, any other gives 2."""
+    from conftest import golden
+    g = golden("ring_order_fp32.json")
+    xs = [np.array(v, np.float32) for v in g["inputs"]]
+    d, _ = to_dev(xs, "f32")
+    y, _ = empty_dev(4, "f32", 4)
+    rc.rc_all_reduce(d, y)
+    yr, _ = empty_dev(4, "f32", 4)
+    rc.rc_ring_all_reduce(d, yr)
+    _sync(rc)
+    for r in range(4):
+        assert to_host(y[r], "f32").tolist() == g["all_reduce_sum"]
+        assert to_host(yr[r], "f32").tolist() == g["all_reduce_sum"]
+
+
+# ------------------------------------------------------------ flat collectives
+CASES = [(1, 37), (2, 64), (3, 1001), (4, 65536), (5, 3), (7, 7777), (8, 65536 + 8 * 13),
+         (8, 2 * 2048 * 8 + 40), (16, 4096 * 16), (16, 33)]
+
+
+@pytest.mark.parametrize("p,n", CASES)
+@pytest.mark.parametrize("dt", DTS)
+def test_all_reduce_reduce_broadcast(rc, p, n, dt):
+    xs = _data(p, n, dt, seed=1000 + p * 7 + n)
+    d, _ = to_dev(xs, dt)
+    for op in OPS:
+        want = oracle.all_reduce(xs, dt, op)
+        y, back = empty_dev(n, dt, p)
+        rc.rc_all_reduce(d, y, op=op)
+        root = (p * 3 + 1) % p
+        yr, back_r = empty_dev(n, dt, 1)
+        rc.rc_reduce(d, yr[0], root=root, op=op)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(y[r], dt), want[r], f"all_reduce {dt} {op} rank {r}")
+        assert_bits(to_host(yr[0], dt), want[0], f"reduce {dt} {op}")
+        check_canary(back, n * ESZ[dt])
+        check_canary(back_r, n * ESZ[dt])
+    # broadcast of rank `root`'s input
+    root = p - 1
+    yb, back_b = empty_dev(n, dt, p)
+    rc.rc_broadcast(d[root], yb, root=root)
+    _sync(rc)
+    for r in range(p):
+        assert_bits(to_host(yb[r], dt), xs[root], f"broadcast {dt} rank {r}")
+    check_canary(back_b, n * ESZ[dt])
+
+
+@pytest.mark.parametrize("p,n", [(1, 40), (2, 64), (3, 999), (4, 65536), (8, 8 * 4104),
+                                 (16, 16 * 2048 + 16 * 3), (5, 5)])
+@pytest.mark.parametrize("in_dt,out_dt", [("f32", "f32"), ("bf16", "bf16"), ("i32", "i32"),
+                                          ("f32", "bf16"), ("bf16", "f32")])
+def test_reduce_scatter_all_gather(rc, p, n, in_dt, out_dt):
+    xs = _data(p, n, in_dt, seed=2000 + p + n)
+    d, _ = to_dev(xs, in_dt)
+    m = n // p
+    for op in OPS:
+        scale = (1.0 / p) if (op == "sum" and in_dt != "i32") else 1.0
+        want = oracle.reduce_scatter(xs, in_dt, out_dt, op, scale)
+        y, back = empty_dev(m, out_dt, p)
+        rc.rc_reduce_scatter(d, y, op=op, scale=scale)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(y[r], out_dt), want[r], f"reduce_scatter {in_dt}->{out_dt} {op} r{r}")
+        check_canary(back, m * ESZ[out_dt])
+        # all_gather of the shards restores the all-reduce (same dtype)
+        ag, back_ag = empty_dev(n, out_dt, p)
+        rc.rc_all_gather(y, ag)
+        _sync(rc)
+        want_ag = oracle.all_gather(want, out_dt)
+        for r in range(p):
+            assert_bits(to_host(ag[r], out_dt), want_ag[r], f"all_gather {out_dt} r{r}")
+        check_canary(back_ag, n * ESZ[out_dt])
+
+
+def test_identity_all_reduce_equals_rs_plus_ag(rc):
+    p, n = 8, 8 * 40960
+    xs = rc_inputs.normal(p, n, seed=5, sigma=1.0)
+    d, _ = to_dev(xs, "f32")
+    ar, _ = empty_dev(n, "f32", p)
+    rs, _ = empty_dev(n // p, "f32", p)
+    ag, _ = empty_dev(n, "f32", p)
+    rc.rc_all_reduce(d, ar)
+    rc.rc_reduce_scatter(d, rs)
+    rc.rc_all_gather(rs, ag)
+    _sync(rc)
+    for r in range(p):
+        assert_bits(to_host(ag[r], "f32"), to_host(ar[r], "f32"), "AR vs RS+AG")
+
+
+# ------------------------------------------------------------ literal ring
+@pytest.mark.parametrize("p,n", [(2, 64), (3, 1001), (4, 65536), (5, 12), (8, 8 * 1024 + 24),
+                                 (16, 16 * 512), (16, 100)])
+@pytest.mark.parametrize("dt", DTS)
+def test_ring_literal(rc, p, n, dt):
+    xs = _data(p, n, dt, seed=3000 + p + n)
+    d, _ = to_dev(xs, dt)
+    for op in OPS:
+        scale = 0.125 if (op == "sum" and dt != "i32") else 1.0
+        want = oracle.ring_all_reduce(xs, dt, op, scale)
+        y, back = empty_dev(n, dt, p)
+        rc.rc_ring_all_reduce(d, y, op=op, scale=scale, variant="literal")
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(y[r], dt), want[r], f"ring {dt} {op} r{r}")
+        check_canary(back, n * ESZ[dt])
+
+
+def test_cfg2_ring_and_oneshot_full_size(rc):
+    """8 ranks x 2,097,152 fp32 ~N(0, 1e-2), seed 1: literal 14-step ring and
+    one-shot, both bit-identical to the oracle's ring simulation."""
+    cfg = rc_inputs.config("cfg2_ring")
+    xs = rc_inputs.draw(cfg)
+    p, n = cfg["p"], cfg["n"]
+    want = oracle.ring_all_reduce(xs, "f32")
+    d, _ = to_dev(xs, "f32")
+    for variant in ("literal", "oneshot"):
+        y, back = empty_dev(n, "f32", p)
+        rc.rc_ring_all_reduce(d, y, variant=variant)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(y[r], "f32"), want[r], f"cfg2 {variant} r{r}")
+        check_canary(back, n * 4)
+
+
+def test_ring_in_place(rc):
+    p, n = 8, 8 * 4096
+    for dt in DTS:
+        xs = _data(p, n, dt, seed=77)
+        want = oracle.ring_all_reduce(xs, dt)
+        d, _ = to_dev(xs, dt)
+        rc.rc_ring_all_reduce(d, d)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(d[r], dt), want[r], f"ring in place {dt} r{r}")
+
+
+# ------------------------------------------------------------ hierarchical
+@pytest.mark.parametrize("p,G,n", [(8, 4, 8 * 1024), (8, 2, 1000), (4, 2, 65536), (16, 4, 4096),
+                                   (6, 3, 999), (8, 1, 512), (8, 8, 512), (2, 2, 10)])
+@pytest.mark.parametrize("dt", DTS)
+def test_hier(rc, p, G, n, dt):
+    xs = _data(p, n, dt, seed=4000 + p * G + n)
+    d, _ = to_dev(xs, dt)
+    for op in OPS:
+        scale = 0.125 if (op == "sum" and dt != "i32") else 1.0
+        want = oracle.hier_all_reduce(xs, G, dt, op, scale)
+        for variant in ("fused", "staged"):
+            y, back = empty_dev(n, dt, p)
+            rc.rc_hier_all_reduce(d, y, G, op=op, scale=scale, variant=variant)
+            _sync(rc)
+            for r in range(p):
+                assert_bits(to_host(y[r], dt), want[r], f"hier {variant} {dt} {op} r{r}")
+            check_canary(back, n * ESZ[dt])
+
+
+def test_cfg3_hier_full_size(rc):
+    """2 groups x 4 ranks, bf16 4,194,304 per rank ~N(0,1), seed 2: fused and
+    staged bit-identical to the oracle's 3-phase simulation; within the fold
+    bound (+1 bf16 ulp) of the flat all-reduce."""
+    cfg = rc_inputs.config("cfg3_hier")
+    xs = rc_inputs.draw(cfg)
+    p, n, G = cfg["p"], cfg["n"], cfg["group"]
+    want = oracle.hier_all_reduce(xs, G, "bf16")
+    d, _ = to_dev(xs, "bf16")
+    for variant in ("fused", "staged"):
+        y, back = empty_dev(n, "bf16", p)
+        rc.rc_hier_all_reduce(d, y, G, variant=variant)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(y[r], "bf16"), want[r], f"cfg3 {variant} r{r}")
+        check_canary(back, n * 2)
+    flat, _ = empty_dev(n, "bf16", 1)
+    rc.rc_reduce(d, flat[0])
+    _sync(rc)
+    hf = oracle.bf16_to_f32(want[0]).astype(np.float64)
+    ff = oracle.bf16_to_f32(to_host(flat[0], "bf16")).astype(np.float64)
+    xa = sum(np.abs(oracle.bf16_to_f32(x).astype(np.float64)) for x in xs)
+    assert np.all(np.abs(hf - ff) <= p * 2.0 ** -24 * xa + np.abs(ff) * 2.0 ** -7 + 2.0 ** -133)
+
+
+# ------------------------------------------------------------ ZeRO-3 layer step
+def test_cfg4_zero3_layer(rc):
+    """Llama-2-7B decoder layer (202,375,168 elements), 8 ranks: all_gather of
+    bf16 parameter shards (compared in full), then reduce_scatter of fp32
+    gradients ~N(0, 1e-3) with scale 1/8 to bf16 (sampled against the oracle,
+    chunk boundaries included)."""
+    p = 8
+    N = rc_inputs.LLAMA2_7B_LAYER_ELEMS
+    m = N // p
+    shards = rc_inputs.draw(rc_inputs.config("cfg4_params"))
+    d, _ = to_dev(shards, "bf16")
+    full, _ = empty_dev(N, "bf16", p, pad_bytes=16)
+    rc.rc_all_gather(d, full)
+    _sync(rc)
+    want = np.concatenate(shards)
+    for r in range(p):
+        assert_bits(to_host(full[r], "bf16"), want, f"cfg4 all_gather r{r}")
+    del full, d, want
+    torch.cuda.empty_cache()
+
+    grads = rc_inputs.draw(rc_inputs.config("cfg4_grads"))
+    g, _ = to_dev(grads, "f32")
+    y, back = empty_dev(m, "bf16", p)
+    rc.rc_reduce_scatter(g, y, in_dtype="f32", out_dtype="bf16", scale=1.0 / p)
+    _sync(rc)
+    rng = np.random.default_rng(4)
+    idx = np.unique(np.concatenate([
+        rng.integers(0, N, 200_000),
+        np.array([c * m + o for c in range(p) for o in (0, 1, 2, 7, 8, m - 9, m - 1)]),
+    ])).astype(np.uint64)
+    ref = oracle.reduce_at(grads, idx, "f32", "bf16", "sum", 1.0 / p)
+    got = np.concatenate([to_host(t, "bf16") for t in y])[idx.astype(np.int64)]
+    assert_bits(got, ref, "cfg4 reduce_scatter (sampled)")
+    check_canary(back, m * 2)
+
+
+# ------------------------------------------------------------ edge cases
+@pytest.mark.parametrize("dt", DTS)
+def test_misaligned_buffers(rc, dt):
+    """Buffers that start off a 16-byte boundary take the scalar path and
+    give the same bits."""
+    p, n = 4, 4 * 1000
+    xs = _data(p, n, dt, seed=9)
+    off = 2 if dt == "bf16" else 4
+    d, _ = to_dev(xs, dt, offset_bytes=off)
+    want = oracle.all_reduce(xs, dt)
+    y, back = empty_dev(n, dt, p, offset_bytes=off)
+    rc.rc_all_reduce(d, y)
+    rs, _ = empty_dev(n // p, dt, p, offset_bytes=off)
+    rc.rc_reduce_scatter(d, rs)
+    ag, _ = empty_dev(n, dt, p, offset_bytes=off)
+    rc.rc_all_gather(rs, ag)
+    ring, _ = empty_dev(n, dt, p, offset_bytes=off)
+    rc.rc_ring_all_reduce(d, ring)
+    hier, _ = empty_dev(n, dt, p, offset_bytes=off)
+    rc.rc_hier_all_reduce(d, hier, 2)
+    _sync(rc)
+    want_h = oracle.hier_all_reduce(xs, 2, dt)
+    for r in range(p):
+        assert_bits(to_host(y[r], dt), want[r], "misaligned all_reduce")
+        assert_bits(to_host(ag[r], dt), want[r], "misaligned rs+ag")
+        assert_bits(to_host(ring[r], dt), want[r], "misaligned ring")
+        assert_bits(to_host(hier[r], dt), want_h[r], "misaligned hier")
+    check_canary(back, off + n * ESZ[dt])
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_special_values(rc, dt):
+    p, n = 8, 8 * 512
+    xs = rc_inputs.special_values(p, n, seed=3, dt=dt)
+    d, _ = to_dev(xs, dt)
+    for op in OPS:
+        want = oracle.all_reduce(xs, dt, op)
+        y, _ = empty_dev(n, dt, p)
+        rc.rc_all_reduce(d, y, op=op)
+        yr, _ = empty_dev(n, dt, p)
+        rc.rc_ring_all_reduce(d, yr, op=op)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(y[r], dt), want[r], f"special {dt} {op}")
+            assert_bits(to_host(yr[r], dt), want[r], f"special ring {dt} {op}")
+
+
+def test_special_int32_wraps(rc):
+    p, n = 4, 4 * 256
+    xs = rc_inputs.special_values(p, n, seed=4, dt="i32")
+    d, _ = to_dev(xs, "i32")
+    for op in OPS:
+        want = oracle.all_reduce(xs, "i32", op)
+        y, _ = empty_dev(n, "i32", p)
+        rc.rc_all_reduce(d, y, op=op)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(y[r], "i32"), want[r], f"int32 {op}")
+
+
+def test_in_place_variants(rc):
+    p, n = 4, 4 * 2048
+    xs = rc_inputs.uniform(p, n, seed=21)
+    want = oracle.all_reduce(xs)
+    d, _ = to_dev(xs, "f32")
+    rc.rc_all_reduce(d, d)                                   # all-reduce in place
+    _sync(rc)
+    for r in range(p):
+        assert_bits(to_host(d[r], "f32"), want[r], "in-place all_reduce")
+    # reduce_scatter whose output is the rank's own slice of its input
+    d2, _ = to_dev(xs, "f32")
+    m = n // p
+    outs = [d2[r][r * m:(r + 1) * m] for r in range(p)]
+    rc.rc_reduce_scatter(d2, outs)
+    _sync(rc)
+    for r in range(p):
+        assert_bits(to_host(outs[r], "f32"), want[r][r * m:(r + 1) * m], "in-place reduce_scatter")
+    # all_gather whose input is the rank's own slot of its output
+    full, _ = to_dev([np.zeros(n, np.float32) for _ in range(p)], "f32")
+    for r in range(p):
+        full[r][r * m:(r + 1) * m].copy_(torch.from_numpy(want[0][r * m:(r + 1) * m]).cuda())
+    rc.rc_all_gather([full[r][r * m:(r + 1) * m] for r in range(p)], full)
+    # reduce into the root's own input, broadcast from a root that is in place
+    d3, _ = to_dev(xs, "f32")
+    rc.rc_reduce(d3, d3[1], root=1)
+    rc.rc_broadcast(d3[1], d3, root=1)
+    # hierarchical in place
+    d4, _ = to_dev(xs, "f32")
+    rc.rc_hier_all_reduce(d4, d4, 2, variant="staged")
+    _sync(rc)
+    want_h = oracle.hier_all_reduce(xs, 2)
+    for r in range(p):
+        assert_bits(to_host(full[r], "f32"), want[0], "in-place all_gather")
+        assert_bits(to_host(d3[r], "f32"), want[0], "in-place reduce+broadcast")
+        assert_bits(to_host(d4[r], "f32"), want_h[r], "in-place hier staged")
+
+
+def test_rejects_bad_buffers_without_launch(rc):
+    from cuda.bindings import runtime as cudart
+    p, n = 4, 1 << 20                 # 4 MiB per rank
+    xs = rc_inputs.uniform(p, n, seed=1)
+    d, _ = to_dev(xs, "f32")
+    y, _ = empty_dev(n, "f32", p)
+    err, base = cudart.cudaMalloc(4 << 20)
+    assert err == cudart.cudaError_t.cudaSuccess
+    try:
+        short = int(base) + (2 << 20)  # only 2 MiB left in its allocation
+        # the pure check must reject it before anything could be launched
+        with pytest.raises(rc.RankCollError):
+            rc.rc_check_buffer(short, n * 4)
+        rc.rc_check_buffer(int(base), n * 4)          # the full allocation is fine
+        before = rc.rc_launch_count()
+        with pytest.raises(rc.RankCollError):         # output runs past its allocation
+            rc.rc_all_reduce(d, [y[0], y[1], y[2], short], n=n)
+        with pytest.raises(rc.RankCollError):         # outputs overlap
+            rc.rc_all_reduce(d, [y[0], y[0], y[2], y[3]])
+        with pytest.raises(rc.RankCollError):         # output overlaps another rank's input
+            rc.rc_all_reduce(d, [y[0], d[0], y[2], y[3]])
+        host = [np.zeros(n, np.float32) for _ in range(p)]
+        with pytest.raises(rc.RankCollError):         # host memory
+            rc.rc_all_reduce([h.ctypes.data for h in host], y, n=n, dtype="f32")
+        _sync(rc)
+        assert rc.rc_launch_count() == before
+    finally:
+        torch.cuda.synchronize()
+        cudart.cudaFree(base)
+
+
+def test_side_stream_and_launch_count(rc):
+    p, n = 8, 8 * 8192
+    xs = rc_inputs.uniform(p, n, seed=2)
+    want = oracle.all_reduce(xs)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        d, _ = to_dev(xs, "f32")
+        y, _ = empty_dev(n, "f32", p)
+        before = rc.rc_launch_count()
+        rc.rc_all_reduce(d, y)
+        assert rc.rc_launch_count() == before + 1
+    rc.rc_stream_status(s)
+    for r in range(p):
+        assert_bits(to_host(y[r], "f32"), want[r], "side stream")
+
+
+def test_bf16_ring_workspace_across_streams(rc):
+    """The bf16 literal ring keeps fp32 partials in the library workspace;
+    calls on two streams in a row see correct results (the second stream
+    waits for the first user's work before reusing it)."""
+    p, n = 8, 8 * 4096
+    xs = rc_inputs.normal(p, n, seed=6, sigma=1.0, dt="bf16")
+    want = oracle.ring_all_reduce(xs, "bf16")
+    d, _ = to_dev(xs, "bf16")
+    outs = []
+    for s in (torch.cuda.Stream(), torch.cuda.Stream()):
+        with torch.cuda.stream(s):
+            y, _ = empty_dev(n, "bf16", p)
+            rc.rc_ring_all_reduce(d, y)
+            outs.append((s, y))
+    for s, y in outs:
+        rc.rc_stream_status(s)
+        for r in range(p):
+            assert_bits(to_host(y[r], "bf16"), want[r], "bf16 ring two streams")
