@@ -8,9 +8,11 @@ seed 1 (the ring / one-shot all-reduce workload), through
   all_reduce (one-shot), reduce_scatter (fp32 -> bf16, scale 1/8),
   all_gather (the bf16 shards), reduce (root 0), broadcast (root 0, in place),
   ring all_reduce (literal 14 steps), hierarchical all_reduce (2 x 4, fused).
-Each collective is timed alone with CUDA events on the launching stream; an
-L2 flush (a 512 MiB write, more than the 126 MB L2) runs between collectives,
-outside the timed events, so every collective reads its inputs from HBM.
+Each collective is timed alone with CUDA events on the launching stream.  An
+L2 flush runs between collectives, outside the timed events: a 512 MiB write
+(more than the 126 MB L2) followed by a 256 MiB read of another buffer, so
+every collective reads its inputs from HBM and starts with an L2 that holds
+no dirty lines of someone else's (the flush's) data to write back.
 
 Effective GB/s = minimum bytes read + written / device time (decimal GB):
   all_reduce p*n*s_in + p*n*s_out; reduce_scatter p*n*s_in + n*s_out;
@@ -46,7 +48,8 @@ UNIT = "GB/s"
 P, N = 8, 2097152
 SEED = 1
 SIGMA = 1e-2
-FLUSH_BYTES = 512 << 20
+FLUSH_BYTES = 512 << 20      # written, then...
+CLEAN_BYTES = 256 << 20      # ...a separate buffer read, so L2 is left holding clean lines
 WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 fp32 "
             "(8 MiB) per rank ~N(0,1e-2) seed 1; step = all_reduce, reduce_scatter fp32->bf16 "
             "x1/8, all_gather bf16, reduce, broadcast, ring all_reduce (literal), "
@@ -223,7 +226,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     ops, _ = step_ops()
-    per_step_budget = max(1.0, 20.0 / max(1, args.steps + args.warmup))
+    per_step_budget = max(0.2, args.ref_seconds / max(1, args.steps + args.warmup))
     # warm-up steps (untimed), then K timed steps, each a bounded sample
     for _ in range(args.warmup):
         cpu_oracle_step_rate(budget_s=0.5 * per_step_budget)
@@ -279,8 +282,12 @@ def run_ours(args):
     y_red = torch.empty(N, dtype=torch.float32, device=dev)
     y_bc = [send[0]] + f32(P - 1)          # root 0 in place
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    cp_a = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
-    cp_b = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def l2_flush():
+        flush.zero_()
+        torch.sum(clean, dim=0, out=sink)
 
     calls = {
         "all_reduce": lambda: rc.rc_all_reduce(send, y_ar),
@@ -291,6 +298,13 @@ def run_ours(args):
         "ring_all_reduce": lambda: rc.rc_ring_all_reduce(send, y_ring, variant="literal"),
         "hier_all_reduce": lambda: rc.rc_hier_all_reduce(send, y_hier, 4, variant="fused"),
     }
+    if args.ops:
+        keep = args.ops.split(",")
+        unknown = set(keep) - set(calls)
+        if unknown:
+            raise SystemExit(f"unknown --ops {sorted(unknown)}")
+        ops = [(nm, b) for nm, b in ops if nm in keep]
+        step_bytes = sum(b for _, b in ops)
     names = [nm for nm, _ in ops]
     K, W = args.steps, args.warmup
     ev = {nm: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -298,7 +312,7 @@ def run_ours(args):
 
     def one_step(k=None):
         for nm in names:
-            flush.zero_()                       # untimed: evicts L2 before each collective
+            l2_flush()                          # untimed: evicts L2 before each collective
             if k is None:
                 calls[nm]()
             else:
@@ -307,20 +321,24 @@ def run_ours(args):
                 calls[nm]()
                 b.record(stream)
 
-    # copy roofline of this library's own copy kernel (same run)
-    for _ in range(3):
-        rc.rc_copy(cp_a, cp_b)
-    cps = []
-    for _ in range(5):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        rc.rc_copy(cp_a, cp_b)
-        b.record(stream)
-        b.synchronize()
-        cps.append(a.elapsed_time(b) * 1e-3)
-    copy_gbs = 2 * (1 << 30) / min(cps) / 1e9
-    del cp_a, cp_b
+    # copy roofline of this library's own copy kernel (same run), 1 GiB
+    copy_gbs = None
+    if not args.no_copy_peak:
+        cp_a = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+        cp_b = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            rc.rc_copy(cp_a, cp_b)
+        cps = []
+        for _ in range(5):
+            l2_flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            rc.rc_copy(cp_a, cp_b)
+            b.record(stream)
+            b.synchronize()
+            cps.append(a.elapsed_time(b) * 1e-3)
+        copy_gbs = 2 * (1 << 30) / min(cps) / 1e9
+        del cp_a, cp_b
 
     for _ in range(W):
         one_step()
@@ -354,6 +372,8 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     e2e_k = max(3, K // 4)
+    if args.no_e2e:
+        e2e_k = 0
 
     def e2e_step():
         for d, h in zip(send, host_in):
@@ -363,16 +383,21 @@ def run_ours(args):
         for h, d in zip(host_out, flat_outs):
             h.copy_(d, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ea.record(stream)
-    for _ in range(e2e_k):
-        e2e_step()
-    eb.record(stream)
-    eb.synchronize()
-    e2e_s, e2e_bytes = reduce_over_ranks(ea.elapsed_time(eb) * 1e-3, step_bytes * e2e_k, world, device=dev)
+    e2e = None
+    if e2e_k:
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        for _ in range(e2e_k):
+            e2e_step()
+        eb.record(stream)
+        eb.synchronize()
+        e2e_s, e2e_bytes = reduce_over_ranks(ea.elapsed_time(eb) * 1e-3, step_bytes * e2e_k, world,
+                                             device=dev)
+        e2e = {"value": round(e2e_bytes / e2e_s / 1e9, 2), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if world > 1:
         import torch.distributed as dist
@@ -388,13 +413,16 @@ def run_ours(args):
         t = per_op_s[nm] / K
         per_op[nm] = {"us": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
                       "frac_of_measured_hbm": round(b / t / 1e9 / peak, 4),
-                      "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4)}
-    t_ar = per_op_s["all_reduce"] / K
-    t_rs = per_op_s["reduce_scatter"] / K
-    per_op["all_reduce"]["busbw_gib_s"] = round(busbw_all_reduce(N * 4, P, t_ar) / 2**30, 1)
-    per_op["reduce_scatter"]["busbw_gib_s"] = round(busbw_reduce_scatter(N * 4, P, t_rs) / 2**30, 1)
-    per_op["ring_all_reduce"]["ring_model_us_at_measured_hbm"] = round(
-        ring_model_seconds(N * 4, P, peak * 1e9) * 1e6, 2)
+                      "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4) if copy_gbs else None}
+    if "all_reduce" in per_op:
+        t_ar = per_op_s["all_reduce"] / K
+        per_op["all_reduce"]["busbw_gib_s"] = round(busbw_all_reduce(N * 4, P, t_ar) / 2**30, 1)
+    if "reduce_scatter" in per_op:
+        t_rs = per_op_s["reduce_scatter"] / K
+        per_op["reduce_scatter"]["busbw_gib_s"] = round(busbw_reduce_scatter(N * 4, P, t_rs) / 2**30, 1)
+    if "ring_all_reduce" in per_op:
+        per_op["ring_all_reduce"]["ring_model_us_at_measured_hbm"] = round(
+            ring_model_seconds(N * 4, P, peak * 1e9) * 1e6, 2)
     dom = max(names, key=lambda nm: per_op_s[nm])
     dom_b = dict(ops)[dom]
     dom_t = per_op_s[dom] / K
@@ -423,10 +451,9 @@ def run_ours(args):
                      "unit": "GB/s", "frac": round(dom_b / dom_t / 1e9 / peak, 4),
                      "traffic": traffic, "algorithmic_bytes": dom_b},
         "per_op": per_op,
-        "copy_kernel_gbs": round(copy_gbs, 1),
+        "copy_kernel_gbs": round(copy_gbs, 1) if copy_gbs else None,
         "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_bytes / e2e_s / 1e9, 2), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk,
     }
@@ -442,6 +469,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=20.0,
+                    help="total CPU budget of the reference arm (warm-up + timed steps)")
+    # profiling aids: time a subset of the step's collectives, skip side phases
+    ap.add_argument("--ops", default="", help="comma-separated subset of the step's collectives")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-copy-peak", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     if args.impl == "reference":

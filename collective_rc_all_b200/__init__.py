@@ -24,6 +24,7 @@ __all__ = [
     "HIER_FUSED", "HIER_STAGED",
     "rc_all_reduce", "rc_reduce_scatter", "rc_all_gather", "rc_reduce", "rc_broadcast",
     "rc_ring_all_reduce", "rc_hier_all_reduce", "rc_copy", "rc_reserve_workspace", "rc_check_buffer",
+    "rc_probe_bounded_wait",
     "rc_stream_status", "rc_launch_count", "rc_finalize", "rc_version", "rc_last_error",
 ]
 
@@ -65,6 +66,7 @@ _decl("rc_hier_all_reduce", [_vpp, _vpp, _i, _i, _sz, _i, _i, _f, _i, _vp])
 _decl("rc_copy", [_vp, _vp, _sz, _vp])
 _decl("rc_reserve_workspace", [_sz, _vp])
 _decl("rc_check_buffer", [_vp, _sz])
+_decl("rc_probe_bounded_wait", [ctypes.c_uint64, _vp])
 _decl("rc_stream_status", [_vp])
 _decl("rc_status_string", [_i], ctypes.c_char_p)
 _decl("rc_last_error", [], ctypes.c_char_p)
@@ -214,6 +216,12 @@ def rc_check_buffer(buf: Buf, nbytes: int) -> None:
     """Raise unless [buf, buf + nbytes) is device memory of the current device
     inside one allocation (no launch)."""
     _check(lib.rc_check_buffer(_addr(buf), int(nbytes)), "rc_check_buffer")
+
+
+def rc_probe_bounded_wait(limit_ns: int, stream=None) -> None:
+    """Launch the failure-path self test (a bounded wait that runs out); the
+    next rc_stream_status on that stream reports the timeout."""
+    _check(lib.rc_probe_bounded_wait(int(limit_ns), _stream(stream)), "rc_probe_bounded_wait")
 
 
 def rc_reserve_workspace(nbytes: int, stream=None):

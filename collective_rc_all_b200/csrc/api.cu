@@ -493,6 +493,12 @@ rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream) 
   return launched(launch_copy(src, dst, bytes, (cudaStream_t)stream), "copy launch");
 }
 
+rc_status rc_probe_bounded_wait(uint64_t limit_ns, rc_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull)
+    return fail(RC_ERR_INVALID_ARG, "limit_ns=%llu outside (0, 1e9]", (unsigned long long)limit_ns);
+  return launched(launch_wait_probe(limit_ns, (cudaStream_t)stream), "wait probe launch");
+}
+
 rc_status rc_check_buffer(const void *ptr, size_t bytes) {
   return check_device_range(ptr, bytes, "buffer", 0);
 }
@@ -509,9 +515,11 @@ rc_status rc_reserve_workspace(size_t bytes, rc_stream_t stream) {
 rc_status rc_stream_status(rc_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "stream");
-  unsigned int timeouts = 0;
+  unsigned int timeouts = 0, fold_timeouts = 0;
   e = read_and_clear_wait_timeouts(&timeouts);
+  if (e == cudaSuccess) e = read_and_clear_fold_timeouts(&fold_timeouts);
   if (e != cudaSuccess) return cuda_fail(e, "status word");
+  timeouts += fold_timeouts;
   if (timeouts) return fail(RC_ERR_TIMEOUT, "%u bounded device wait(s) gave up", timeouts);
   return RC_OK;
 }

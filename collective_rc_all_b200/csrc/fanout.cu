@@ -31,9 +31,10 @@ __device__ unsigned int g_wait_timeouts = 0;
 
 namespace {
 
-constexpr uint32_t kTile = 32 * 1024;  // bytes per stage
+constexpr uint32_t kMaxTile = 32 * 1024;  // bytes per stage, at most
+constexpr uint32_t kMinTile = 4 * 1024;
 constexpr int kStages = 6;
-constexpr int kLookahead = 4;          // loads in flight ahead of the stores
+constexpr int kLookahead = 4;             // loads in flight ahead of the stores
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 static_assert(kLookahead <= kStages - 1, "a stage must be free when its load is issued");
 
@@ -44,10 +45,11 @@ struct FanoutParams {
   uint64_t src_bytes;
   uint64_t tiles_per_src;
   uint64_t units;            // nsrc * tiles_per_src
+  uint32_t tile;             // bytes per unit (a power of two in [4 KiB, 32 KiB])
   int p;
 };
 
-__global__ void __launch_bounds__(32) fanout_bulk_kernel(const __grid_constant__ FanoutParams a) {
+__global__ void __launch_bounds__(32) rc_fanout_bulk_kernel(const __grid_constant__ FanoutParams a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t bars[kStages];
   if (threadIdx.x != 0) return;
@@ -60,11 +62,12 @@ __global__ void __launch_bounds__(32) fanout_bulk_kernel(const __grid_constant__
   const uint64_t u1 = a.units * (blockIdx.x + 1) / G;
   const int64_t K = (int64_t)(u1 - u0);
 
+  const uint32_t tile = a.tile;
   auto unit_bytes = [&](uint64_t u, uint64_t &src_idx, uint64_t &off) -> uint32_t {
     src_idx = u / a.tiles_per_src;
-    off = (u - src_idx * a.tiles_per_src) * kTile;
+    off = (u - src_idx * a.tiles_per_src) * tile;
     const uint64_t rem = a.src_bytes - off;
-    return (uint32_t)(rem < kTile ? rem : kTile);
+    return (uint32_t)(rem < tile ? rem : tile);
   };
 
   bool failed = false;
@@ -76,7 +79,7 @@ __global__ void __launch_bounds__(32) fanout_bulk_kernel(const __grid_constant__
       uint64_t r, off;
       const uint32_t bytes = unit_bytes(u0 + k, r, off);
       mbar_arrive_expect_tx(&bars[s], bytes);
-      bulk_load(smem + (size_t)s * kTile, a.src[r] + off, bytes, &bars[s]);
+      bulk_load(smem + (size_t)s * tile, a.src[r] + off, bytes, &bars[s]);
       ++loads_issued;
     }
     const int64_t j = k - kLookahead;
@@ -90,10 +93,10 @@ __global__ void __launch_bounds__(32) fanout_bulk_kernel(const __grid_constant__
       fence_proxy_async_smem();
       uint64_t r, off;
       const uint32_t bytes = unit_bytes(u0 + j, r, off);
-      const unsigned char *tile = smem + (size_t)s * kTile;
+      const unsigned char *buf = smem + (size_t)s * tile;
       for (int q = 0; q < a.p; ++q) {
         if ((a.skip[q] >> r) & 1u) continue;
-        bulk_store(a.dst[q] + r * a.src_bytes + off, tile, bytes);
+        bulk_store(a.dst[q] + r * a.src_bytes + off, buf, bytes);
       }
       bulk_commit();
     }
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(32) fanout_bulk_kernel(const __grid_constant__
 // Fallback for buffers that are not 16-byte aligned (or sizes not a multiple
 // of 16 bytes): element copies, blockIdx.y = destination rank, x grid-stride.
 template <typename E>
-__global__ void fanout_elem_kernel(const __grid_constant__ FanoutParams a, int nsrc) {
+__global__ void rc_fanout_elem_kernel(const __grid_constant__ FanoutParams a, int nsrc) {
   const int q = blockIdx.y;
   const uint64_t per_src = a.src_bytes / sizeof(E);
   const uint64_t total = per_src * nsrc;
@@ -125,7 +128,24 @@ __global__ void fanout_elem_kernel(const __grid_constant__ FanoutParams a, int n
   }
 }
 
+// Exercises the bounded-wait path: waits on a barrier phase that nothing will
+// complete, gives up after limit_ns and records the timeout like any other
+// wait of this library.  No copy is in flight, so returning is safe.
+__global__ void rc_wait_probe_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  mbar_init_fence();
+  if (!mbar_wait_bounded(&bar, 0, limit_ns)) atomicAdd(&g_wait_timeouts, 1u);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s) {
+  rc_wait_probe_kernel<<<1, 32, 0, s>>>(limit_ns);
+  note_launches(1);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s) {
   FanoutParams a{};
@@ -145,29 +165,42 @@ cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s) {
   cudaError_t err;
   const int sms = device_sm_count();
   if (aligned) {
-    a.tiles_per_src = (job.src_bytes + kTile - 1) / kTile;
+    // tile: the largest power of two <= 32 KiB that still gives every SM about
+    // four units, so small fan-outs still pipeline
+    const uint64_t total = job.src_bytes * job.nsrc;
+    uint32_t tile = kMaxTile;
+    while (tile > kMinTile && total / tile < 4ull * sms) tile >>= 1;
+    tile = (uint32_t)env_int("RC_FANOUT_TILE", (int)tile);
+    if (tile < 16 || tile % 16 || tile > kMaxTile) tile = kMaxTile;
+    a.tile = tile;
+    a.tiles_per_src = (job.src_bytes + tile - 1) / tile;
     a.units = a.tiles_per_src * job.nsrc;
-    const size_t smem = (size_t)kStages * kTile;
+    const size_t smem = (size_t)kStages * tile;
     static std::atomic<uint64_t> attr_set{0};  // one bit per device
     int dev = 0;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_set.load() & bit)) {
-      err = cudaFuncSetAttribute(fanout_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
+      err = cudaFuncSetAttribute(rc_fanout_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(kStages * kMaxTile));
       if (err != cudaSuccess) return err;
       attr_set.fetch_or(bit);
     }
-    const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(sms, a.units));
-    fanout_bulk_kernel<<<(unsigned)grid, 32, smem, s>>>(a);
+    int occ = 0;
+    if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rc_fanout_bulk_kernel, 32, smem)) !=
+        cudaSuccess)
+      return err;
+    occ = std::max(1, std::min(occ, env_int("RC_FANOUT_CTAS_PER_SM", 8)));
+    const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>((uint64_t)sms * occ, a.units));
+    rc_fanout_bulk_kernel<<<(unsigned)grid, 32, smem, s>>>(a);
   } else {
     const uint64_t per_src = job.src_bytes / job.elem_bytes;
     const uint64_t total = per_src * job.nsrc;
     const unsigned gx = (unsigned)std::max<uint64_t>(
         1, std::min<uint64_t>((total + 255) / 256, (uint64_t)sms * 4));
     dim3 grid(gx, job.p);
-    if (job.elem_bytes == 2) fanout_elem_kernel<uint16_t><<<grid, 256, 0, s>>>(a, job.nsrc);
-    else fanout_elem_kernel<uint32_t><<<grid, 256, 0, s>>>(a, job.nsrc);
+    if (job.elem_bytes == 2) rc_fanout_elem_kernel<uint16_t><<<grid, 256, 0, s>>>(a, job.nsrc);
+    else rc_fanout_elem_kernel<uint32_t><<<grid, 256, 0, s>>>(a, job.nsrc);
   }
   note_launches(1);
   return cudaGetLastError();

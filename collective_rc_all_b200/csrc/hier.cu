@@ -39,7 +39,7 @@ struct HierParams {
 };
 
 template <int PMAX, class T, int OP, bool VECTOR>
-__global__ void __launch_bounds__(kNT) hier_fused_kernel(const __grid_constant__ HierParams a) {
+__global__ void __launch_bounds__(kNT) rc_hier_reg_kernel(const __grid_constant__ HierParams a) {
   using Acc = typename T::Acc;
   constexpr int VEC = VECTOR ? kVec<T> : 1;
   const int p = a.p, G = a.G, ng = a.ng;
@@ -131,7 +131,7 @@ cudaError_t run_fused(const HierJob &job, cudaStream_t s) {
   }
   constexpr int VEC = kVec<T>;
   const bool vector = aligned && a.CG % VEC == 0 && a.CL % VEC == 0 && a.n % VEC == 0;
-  auto kern = vector ? hier_fused_kernel<PMAX, T, OP, true> : hier_fused_kernel<PMAX, T, OP, false>;
+  auto kern = vector ? rc_hier_reg_kernel<PMAX, T, OP, true> : rc_hier_reg_kernel<PMAX, T, OP, false>;
   a.units = vector ? a.n / VEC : a.n;
   int occ = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNT, 0);
@@ -164,6 +164,22 @@ cudaError_t fused_by_op(const HierJob &job, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s) {
+  FoldJob f{};
+  f.p = job.p;
+  f.G = job.G;
+  f.n = job.n;
+  f.CG = (job.n + job.G - 1) / job.G;
+  f.CL = (job.n + job.p / job.G - 1) / (job.p / job.G);
+  f.in_dt = f.out_dt = job.dt;
+  f.op = job.op;
+  f.scale = job.scale;
+  f.mode = kModeAll;
+  f.ndst = job.p;
+  for (int r = 0; r < job.p; ++r) {
+    f.src[r] = job.x[r];
+    f.dst[r] = job.y[r];
+  }
+  if (fold_tma_eligible(f)) return launch_fold_tma(f, s);
   switch (job.dt) {
     case kF32: return fused_by_op<F32>(job, s);
     case kBF16: return fused_by_op<BF16>(job, s);

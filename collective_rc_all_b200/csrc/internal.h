@@ -28,6 +28,19 @@ struct ReduceJob {
   int ndst;  // kModeAll: number of outputs (0 means p)
 };
 
+// A p-source fold over aligned 16-byte vectors (fold.cu).  G = p is the flat
+// ring order (CG = ceil(n/p), CL = n); G < p is the hierarchical order.
+struct FoldJob {
+  const void *src[kMaxP];
+  void *dst[kMaxP];
+  int p, G;
+  uint64_t n, CG, CL;
+  int in_dt, out_dt, op;
+  float scale;
+  int mode;
+  int ndst;  // outputs in kModeAll
+};
+
 struct FanoutJob {
   const void *src[kMaxP];  // nsrc sources of src_bytes each
   void *dst[kMaxP];        // p destinations; source r lands at dst[q] + r * src_bytes
@@ -59,11 +72,16 @@ struct HierJob {
 };
 
 cudaError_t launch_reduce(const ReduceJob &job, cudaStream_t s);
+bool fold_tma_eligible(const FoldJob &job);
+cudaError_t launch_fold_tma(const FoldJob &job, cudaStream_t s);
+cudaError_t read_and_clear_fold_timeouts(unsigned int *count);
 cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s);
 cudaError_t launch_ring_literal(const RingJob &job, cudaStream_t s);
 cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s);
 cudaError_t launch_hier_staged(const HierJob &job, cudaStream_t s);
 cudaError_t launch_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);
+
+cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s);
 
 // Device-side bounded waits report here (fanout.cu).
 cudaError_t read_and_clear_wait_timeouts(unsigned int *count);

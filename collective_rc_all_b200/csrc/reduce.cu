@@ -52,7 +52,7 @@ __device__ __forceinline__ int rot(uint64_t c, int k, int p) {
 }
 
 template <int PMAX, class TI, class TO, int OP, bool VECTOR>
-__global__ void __launch_bounds__(kNT) reduce_kernel(const __grid_constant__ ReduceParams a) {
+__global__ void __launch_bounds__(kNT) rc_reduce_reg_kernel(const __grid_constant__ ReduceParams a) {
   using Acc = typename TI::Acc;
   constexpr int VEC = VECTOR ? kVec<TI> : 1;
   constexpr int ILP = VECTOR ? ilp_for<PMAX>() : 1;
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kNT) reduce_kernel(const __grid_constant__ Red
 // Elements past the last whole vector (n % VEC of them, all in the last
 // chunk) -- one small CTA, scalar.
 template <int PMAX, class TI, class TO, int OP>
-__global__ void __launch_bounds__(32) reduce_tail_kernel(const __grid_constant__ ReduceParams a,
+__global__ void __launch_bounds__(32) rc_reduce_tail_kernel(const __grid_constant__ ReduceParams a,
                                                           uint64_t first) {
   using Acc = typename TI::Acc;
   const int p = a.p;
@@ -189,8 +189,33 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
 
   const int sms = device_sm_count();
   cudaError_t err;
+  FoldJob f{};
+  f.p = p;
+  f.G = p;
+  f.n = n;
+  f.CG = C;
+  f.CL = n;
+  f.in_dt = job.in_dt;
+  f.out_dt = job.out_dt;
+  f.op = job.op;
+  f.scale = job.scale;
+  f.mode = job.mode;
+  f.ndst = a.ndst;
+  for (int r = 0; r < p; ++r) f.src[r] = job.src[r];
+  for (int r = 0; r < ndst; ++r) f.dst[r] = job.dst[r];
+  if (vector && fold_tma_eligible(f)) {
+    // the staged fold covers whole vectors; the tail (n % VEC elements) is scalar
+    if ((err = launch_fold_tma(f, s)) != cudaSuccess) return err;
+    a.nvec = n / VEC;
+    if (a.nvec * VEC < n) {
+      rc_reduce_tail_kernel<PMAX, TI, TO, OP><<<1, 32, 0, s>>>(a, a.nvec * VEC);
+      note_launches(1);
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+  }
   if (vector) {
-    auto kern = reduce_kernel<PMAX, TI, TO, OP, true>;
+    auto kern = rc_reduce_reg_kernel<PMAX, TI, TO, OP, true>;
     int occ = 0;
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNT, 0);
     if (err != cudaSuccess) return err;
@@ -205,12 +230,12 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
       if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
     if (a.nvec * VEC < n) {
-      reduce_tail_kernel<PMAX, TI, TO, OP><<<1, 32, 0, s>>>(a, a.nvec * VEC);
+      rc_reduce_tail_kernel<PMAX, TI, TO, OP><<<1, 32, 0, s>>>(a, a.nvec * VEC);
       note_launches(1);
       if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
   } else {
-    auto kern = reduce_kernel<PMAX, TI, TO, OP, false>;
+    auto kern = rc_reduce_reg_kernel<PMAX, TI, TO, OP, false>;
     int occ = 0;
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNT, 0);
     if (err != cudaSuccess) return err;

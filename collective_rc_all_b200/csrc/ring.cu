@@ -26,8 +26,10 @@
 // the same thread stored at step k, so program order is the only
 // synchronisation -- no grid barrier, no flags, nothing can wait forever.
 // Within one step the ranks' reads and writes touch disjoint locations, so a
-// thread issues the loads of a group of RG ranks before any of their stores
-// (memory-level parallelism) without changing the schedule's result.
+// thread issues all loads of a step before its stores, and it loads the next
+// step's x values (independent of the partials) while the current step folds:
+// only the partials' round trip through L2 stays on the dependent chain.  The
+// per-(step, rank) chunk addresses come from a table in shared memory.
 #include <algorithm>
 #include <type_traits>
 
@@ -87,6 +89,25 @@ __device__ __forceinline__ void load_in(const char *p, typename T::Acc (&a)[VEC]
   }
 }
 
+// input element(s) of type T in their stored form (16-byte vector or one element)
+template <class T, int VEC>
+__device__ __forceinline__ typename std::conditional<(VEC > 1), uint4, uint32_t>::type load_raw(
+    const char *p) {
+  if constexpr (VEC > 1) return ld_cg_v4(p);
+  else if constexpr (T::kBytes == 2) return ld_cg_u16(p);
+  else return ld_cg_u32(p);
+}
+template <class T, int VEC>
+__device__ __forceinline__ void unpack_raw(const uint4 &raw, typename T::Acc (&a)[VEC]) {
+  unpack<T>(raw, a);
+}
+template <class T, int VEC>
+__device__ __forceinline__ void unpack_raw(uint32_t raw, typename T::Acc (&a)[VEC]) {
+  if constexpr (std::is_same<T, BF16>::value) a[0] = bf16_bits_to_f32(raw);
+  else if constexpr (std::is_same<T, F32>::value) a[0] = __uint_as_float(raw);
+  else a[0] = (int32_t)raw;
+}
+
 // partial (raw 32-bit accumulators) load / store
 template <class Acc, int VEC>
 __device__ __forceinline__ void load_part(const char *p, Acc (&a)[VEC]) {
@@ -136,110 +157,152 @@ __device__ __forceinline__ void store_out(char *p, const typename T::Acc (&a)[VE
 
 __device__ __forceinline__ int mod_p(int v, int p) { return v < 0 ? v + p : v; }
 
-template <class T, int OP, bool VECTOR, int RG>
-__global__ void __launch_bounds__(kRingNT) ring_literal_kernel(const __grid_constant__ RingParams a) {
+// Chunk addresses of every (step, rank) of the schedule, computed once per
+// thread block; a thread adds its own offset inside the chunk.
+struct RsEntry {      // reduce-scatter step k, sender r -> receiver d = r+1
+  const char *msg;    // k == 0: x_r at chunk c (input stride); else r's partial (4-byte stride)
+  const char *own;    // x_d at chunk c (input stride)
+  char *dst;          // d's partial (4-byte stride), or y_d at chunk d on the last step
+  uint64_t len;       // elements in chunk c
+};
+struct AgEntry {      // all-gather step k, r -> d = r+1, chunk c = r-k
+  const char *src;
+  char *dst;
+  uint64_t len;
+};
+
+// Registers are capped so that at least 4 (PMAX <= 8) or 2 (PMAX = 16) thread
+// blocks fit per SM: a typical launch then keeps every offset resident at
+// once, instead of running a second full 2(p-1)-step chain for a few blocks.
+template <class T, int OP, bool VECTOR, int PMAX>
+__global__ void __launch_bounds__(kRingNT, (PMAX <= 8 ? 4 : 2))
+    rc_ring_literal_kernel(const __grid_constant__ RingParams a) {
   using Acc = typename T::Acc;
   constexpr int VEC = VECTOR ? kVec<T> : 1;
+  using Raw = typename std::conditional<VECTOR, uint4, uint32_t>::type;
+  constexpr int RG = 4;  // ranks folded together (register budget)
   constexpr bool kWs = std::is_same<T, BF16>::value;  // bf16: fp32 partials in workspace
+  constexpr int kIn = T::kBytes;
+  __shared__ RsEntry rs[kMaxRanks - 1][PMAX];
+  __shared__ AgEntry ag[kMaxRanks - 1][PMAX];
   const int p = a.p;
   const uint64_t C = a.C;
 
-  auto chunk_len = [&](int c) -> uint64_t {
-    const uint64_t b = (uint64_t)c * C;
-    return b >= a.n ? 0 : (a.n - b < C ? a.n - b : C);
-  };
-  // where rank `rank` keeps its partial of chunk c for step parity `par`
-  auto part = [&](int rank, int c, int par, uint64_t oe) -> char * {
-    if constexpr (kWs) return a.ws + (((uint64_t)(par * p + rank)) * C + oe) * 4;
-    else return a.y[rank] + ((uint64_t)c * C + oe) * 4;
-  };
+  for (int i = threadIdx.x; i < (p - 1) * p; i += blockDim.x) {
+    const int k = i / p, r = i - k * p;
+    const int d = (r + 1 < p) ? r + 1 : 0;
+    // reduce-scatter entry
+    {
+      const int c = mod_p(r - k - 1, p);
+      const uint64_t b = (uint64_t)c * C;
+      RsEntry e;
+      e.len = b >= a.n ? 0 : (a.n - b < C ? a.n - b : C);
+      e.own = a.x[d] + b * kIn;
+      if (k == 0) e.msg = a.x[r] + b * kIn;
+      else if (kWs) e.msg = a.ws + ((uint64_t)(((k - 1) & 1) * p + r)) * C * 4;
+      else e.msg = a.y[r] + b * 4;
+      if (k == p - 2) e.dst = a.y[d] + b * kIn;
+      else if (kWs) e.dst = a.ws + ((uint64_t)((k & 1) * p + d)) * C * 4;
+      else e.dst = a.y[d] + b * 4;
+      rs[k][r] = e;
+    }
+    // all-gather entry
+    {
+      const int c = mod_p(r - k, p);
+      const uint64_t b = (uint64_t)c * C;
+      AgEntry e;
+      e.len = b >= a.n ? 0 : (a.n - b < C ? a.n - b : C);
+      e.src = a.y[r] + b * kIn;
+      e.dst = a.y[d] + b * kIn;
+      ag[k][r] = e;
+    }
+  }
+  __syncthreads();
 
   const uint64_t G = gridDim.x;
   const uint64_t o0 = a.units * blockIdx.x / G;
   const uint64_t o1 = a.units * (blockIdx.x + 1) / G;
 
   for (uint64_t o = o0 + threadIdx.x; o < o1; o += blockDim.x) {
-    const uint64_t oe = o * VEC;  // element offset inside every chunk
+    const uint64_t oe = o * VEC;                 // element offset inside every chunk
+    const uint64_t oin = oe * kIn, o4 = oe * 4;  // byte offsets: input / partial
 
-    // ---- phase 1: reduce-scatter, p-1 steps
+    // ---- phase 1: reduce-scatter, p-1 steps.  own[] holds the receivers' x_d
+    // of the current step in input form, loaded one step ahead.
+    Raw own[PMAX], nxt[PMAX];
+#pragma unroll
+    for (int r = 0; r < PMAX; ++r)
+      if (r < p && oe < rs[0][r].len) own[r] = load_raw<T, VEC>(rs[0][r].own + oin);
     for (int k = 0; k + 1 < p; ++k) {
       const bool last = (k + 2 == p);
-      for (int r0 = 0; r0 < p; r0 += RG) {
-        Acc msg[RG][VEC], own[RG][VEC];
-        bool act[RG];
+      if (!last) {  // next step's x_d, in flight while this step folds
 #pragma unroll
-        for (int g = 0; g < RG; ++g) {  // all sends/receives' loads first
+        for (int r = 0; r < PMAX; ++r)
+          if (r < p && oe < rs[k + 1][r].len) nxt[r] = load_raw<T, VEC>(rs[k + 1][r].own + oin);
+      }
+#pragma unroll
+      for (int r0 = 0; r0 < PMAX; r0 += RG) {
+        if (r0 >= p) break;
+        Acc msg[RG][VEC];
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {  // the sends of this group of ranks
           const int r = r0 + g;
-          act[g] = false;
-          if (r < p) {
-            const int c = mod_p(r - k - 1, p);
-            const int d = (r + 1 < p) ? r + 1 : 0;
-            if (oe < chunk_len(c)) {
-              act[g] = true;
-              const uint64_t e = (uint64_t)c * C + oe;
-              if (k == 0) load_in<T, VEC>(a.x[r] + e * T::kBytes, msg[g]);
-              else load_part<Acc, VEC>(part(r, c, (k - 1) & 1, oe), msg[g]);
-              load_in<T, VEC>(a.x[d] + e * T::kBytes, own[g]);
+          if (r < p && oe < rs[k][r].len) {
+            if (k == 0) unpack_raw<T, VEC>(load_raw<T, VEC>(rs[0][r].msg + oin), msg[g]);
+            else load_part<Acc, VEC>(rs[k][r].msg + o4, msg[g]);
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {  // the receives
+          const int r = r0 + g;
+          if (r < p && oe < rs[k][r].len) {
+            Acc x[VEC];
+            unpack_raw<T, VEC>(own[r], x);
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) msg[g][j] = combine<OP>(msg[g][j], x[j]);
+            if (last) {  // receiver d now owns the finished chunk c (== d)
+#pragma unroll
+              for (int j = 0; j < VEC; ++j) msg[g][j] = finish<OP>(msg[g][j], a.scale);
+              store_out<T, VEC>(rs[k][r].dst + oin, msg[g]);
+            } else {
+              store_part<Acc, VEC>(rs[k][r].dst + o4, msg[g]);
             }
           }
         }
+      }
+      if (!last) {
 #pragma unroll
-        for (int g = 0; g < RG; ++g) {  // then the folds and stores
-          if (!act[g]) continue;
-          const int r = r0 + g;
-          const int c = mod_p(r - k - 1, p);
-          const int d = (r + 1 < p) ? r + 1 : 0;
-#pragma unroll
-          for (int j = 0; j < VEC; ++j) msg[g][j] = combine<OP>(msg[g][j], own[g][j]);
-          if (last) {  // receiver d now owns the finished chunk c (== d)
-#pragma unroll
-            for (int j = 0; j < VEC; ++j) msg[g][j] = finish<OP>(msg[g][j], a.scale);
-            store_out<T, VEC>(a.y[d] + ((uint64_t)c * C + oe) * T::kBytes, msg[g]);
-          } else {
-            store_part<Acc, VEC>(part(d, c, k & 1, oe), msg[g]);
-          }
-        }
+        for (int r = 0; r < PMAX; ++r) own[r] = nxt[r];
       }
     }
 
     // ---- phase 2: all-gather, p-1 steps, the receiver overwrites
     for (int k = 0; k + 1 < p; ++k) {
-      for (int r0 = 0; r0 < p; r0 += RG) {
-        uint4 v16[RG];
-        uint32_t v4[RG];
-        bool act[RG];
+      uint4 v16[PMAX];
+      uint32_t v4[PMAX];
 #pragma unroll
-        for (int g = 0; g < RG; ++g) {
-          const int r = r0 + g;
-          act[g] = false;
-          if (r < p) {
-            const int c = mod_p(r - k, p);
-            if (oe < chunk_len(c)) {
-              act[g] = true;
-              const char *src = a.y[r] + ((uint64_t)c * C + oe) * T::kBytes;
-              if constexpr (VECTOR) v16[g] = ld_cg_v4(src);
-              else if constexpr (T::kBytes == 2) v4[g] = ld_cg_u16(src);
-              else v4[g] = ld_cg_u32(src);
-            }
-          }
+      for (int r = 0; r < PMAX; ++r) {
+        if (r < p && oe < ag[k][r].len) {
+          const char *src = ag[k][r].src + oin;
+          if constexpr (VECTOR) v16[r] = ld_cg_v4(src);
+          else if constexpr (kIn == 2) v4[r] = ld_cg_u16(src);
+          else v4[r] = ld_cg_u32(src);
         }
+      }
 #pragma unroll
-        for (int g = 0; g < RG; ++g) {
-          if (!act[g]) continue;
-          const int r = r0 + g;
-          const int c = mod_p(r - k, p);
-          const int d = (r + 1 < p) ? r + 1 : 0;
-          char *dst = a.y[d] + ((uint64_t)c * C + oe) * T::kBytes;
-          if constexpr (VECTOR) st_v4(dst, v16[g]);
-          else if constexpr (T::kBytes == 2) st_u16(dst, v4[g]);
-          else st_u32(dst, v4[g]);
+      for (int r = 0; r < PMAX; ++r) {
+        if (r < p && oe < ag[k][r].len) {
+          char *dst = ag[k][r].dst + oin;
+          if constexpr (VECTOR) st_v4(dst, v16[r]);
+          else if constexpr (kIn == 2) st_u16(dst, v4[r]);
+          else st_u32(dst, v4[r]);
         }
       }
     }
   }
 }
 
-template <class T, int OP>
+template <class T, int OP, int PMAX>
 cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   RingParams a{};
   const int p = job.p;
@@ -257,9 +320,8 @@ cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   }
   constexpr int VEC = kVec<T>;
   const bool vector = aligned && a.C % VEC == 0 && a.n % VEC == 0;
-  constexpr int RG = std::is_same<T, BF16>::value ? 4 : 8;
   const int sms = device_sm_count();
-  auto kern = vector ? ring_literal_kernel<T, OP, true, RG> : ring_literal_kernel<T, OP, false, RG>;
+  auto kern = vector ? rc_ring_literal_kernel<T, OP, true, PMAX> : rc_ring_literal_kernel<T, OP, false, PMAX>;
   a.units = vector ? a.C / VEC : a.C;
   int occ = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kRingNT, 0);
@@ -272,12 +334,19 @@ cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <class T, int OP>
+cudaError_t ring_by_p(const RingJob &job, cudaStream_t s) {
+  if (job.p <= 4) return run_ring<T, OP, 4>(job, s);
+  if (job.p <= 8) return run_ring<T, OP, 8>(job, s);
+  return run_ring<T, OP, 16>(job, s);
+}
+
 template <class T>
 cudaError_t ring_by_op(const RingJob &job, cudaStream_t s) {
   switch (job.op) {
-    case kSum: return run_ring<T, kSum>(job, s);
-    case kMax: return run_ring<T, kMax>(job, s);
-    case kMin: return run_ring<T, kMin>(job, s);
+    case kSum: return ring_by_p<T, kSum>(job, s);
+    case kMax: return ring_by_p<T, kMax>(job, s);
+    case kMin: return ring_by_p<T, kMin>(job, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -190,6 +190,13 @@ rc_status rc_reserve_workspace(size_t bytes, rc_stream_t stream);
  * since the last call (the flag is cleared), else RC_OK. */
 rc_status rc_stream_status(rc_stream_t stream);
 
+/* Failure-path self test: launches one kernel whose single thread waits on a
+ * barrier phase that nothing completes.  The wait is bounded like every wait
+ * in this library: after limit_ns (0 < limit_ns <= 1e9) it gives up, records
+ * the event and returns, so the context stays usable and the next
+ * rc_stream_status(stream) returns RC_ERR_TIMEOUT. */
+rc_status rc_probe_bounded_wait(uint64_t limit_ns, rc_stream_t stream);
+
 /* Static description of a status code. */
 const char *rc_status_string(rc_status status);
 

@@ -442,3 +442,76 @@ def test_bf16_ring_workspace_across_streams(rc):
         rc.rc_stream_status(s)
         for r in range(p):
             assert_bits(to_host(y[r], "bf16"), want[r], "bf16 ring two streams")
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(rc):
+    """A device wait that runs out returns an error status to the host; the
+    context stays usable and the next collective is still correct."""
+    rc.rc_stream_status()                       # clear anything earlier
+    rc.rc_probe_bounded_wait(20_000_000)        # 20 ms, nothing will arrive
+    with pytest.raises(rc.RankCollError) as e:
+        rc.rc_stream_status()
+    assert e.value.status == 4
+    rc.rc_stream_status()                       # the flag was cleared
+    p, n = 4, 4096
+    xs = rc_inputs.uniform(p, n, seed=8)
+    d, _ = to_dev(xs, "f32")
+    y, _ = empty_dev(n, "f32", p)
+    rc.rc_all_reduce(d, y)
+    _sync(rc)
+    want = oracle.all_reduce(xs)
+    for r in range(p):
+        assert_bits(to_host(y[r], "f32"), want[r], "after timeout")
+
+
+@pytest.mark.parametrize("dt", DTS)
+def test_register_path_matches_oracle(rc, dt, monkeypatch):
+    """The register-only fold (used when the bulk-copy path is not eligible)
+    gives the same bits as the oracle; forced here on aligned data."""
+    monkeypatch.setenv("RC_NO_TMA_FOLD", "1")
+    p, n = 8, 8 * 4096 + 8 * 24
+    xs = _data(p, n, dt, seed=31)
+    d, _ = to_dev(xs, dt)
+    for op in OPS:
+        y, _ = empty_dev(n, dt, p)
+        rc.rc_all_reduce(d, y, op=op)
+        rs, _ = empty_dev(n // p, dt, p)
+        rc.rc_reduce_scatter(d, rs, op=op)
+        h, _ = empty_dev(n, dt, p)
+        rc.rc_hier_all_reduce(d, h, 4, op=op)
+        _sync(rc)
+        want = oracle.all_reduce(xs, dt, op)
+        want_h = oracle.hier_all_reduce(xs, 4, dt, op)
+        for r in range(p):
+            assert_bits(to_host(y[r], dt), want[r], f"register all_reduce {dt} {op}")
+            assert_bits(to_host(h[r], dt), want_h[r], f"register hier {dt} {op}")
+        assert_bits(np.concatenate([to_host(t, dt) for t in rs]), want[0], f"register rs {dt} {op}")
+
+
+@pytest.mark.parametrize("tile", ["4096", "16384"])
+def test_fanout_tile_sizes(rc, tile, monkeypatch):
+    """The fan-out gives the same bytes whatever its tile size (ragged last tile)."""
+    monkeypatch.setenv("RC_FANOUT_TILE", tile)
+    p, m = 8, 12345 * 8
+    shards = rc_inputs.uniform(p, m, seed=12, dt="bf16")
+    d, _ = to_dev(shards, "bf16")
+    y, back = empty_dev(p * m, "bf16", p)
+    rc.rc_all_gather(d, y)
+    b, back_b = empty_dev(m, "bf16", p)
+    rc.rc_broadcast(d[3], b, root=3)
+    _sync(rc)
+    for r in range(p):
+        assert_bits(to_host(y[r], "bf16"), np.concatenate(shards), "all_gather tile")
+        assert_bits(to_host(b[r], "bf16"), shards[3], "broadcast tile")
+    check_canary(back, p * m * 2)
+    check_canary(back_b, m * 2)
+
+
+@pytest.mark.parametrize("nbytes", [16, 1000, 1 << 20, (1 << 24) + 48])
+def test_copy_kernel(rc, nbytes):
+    a = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device="cuda")
+    b = torch.zeros(nbytes + 64, dtype=torch.uint8, device="cuda")
+    rc.rc_copy(a, b, nbytes)
+    _sync(rc)
+    assert torch.equal(a, b[:nbytes])
+    assert int(b[nbytes:].sum()) == 0
