@@ -106,7 +106,9 @@ __device__ __forceinline__ int fold_rank(int k, int cg, int cl, int G, int ng) {
   return gg * G + m;
 }
 
-template <int PMAX, class TI, class TO, int OP>
+// GROUPED = false: the flat fold (G = p), a plain left-to-right fold;
+// GROUPED = true: the hierarchical fold with group boundaries.
+template <int PMAX, class TI, class TO, int OP, bool GROUPED>
 __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_constant__ FoldParams a) {
   using Acc = typename TI::Acc;
   constexpr int VEC = kVec<TI>;
@@ -144,6 +146,7 @@ __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_co
 
   const uint64_t Gd = gridDim.x;
   const int64_t K = a.ntiles > blockIdx.x ? (int64_t)((a.ntiles - blockIdx.x + Gd - 1) / Gd) : 0;
+  const uint32_t tv = a.tv, tile_bytes = a.tile_bytes, stage_bytes = a.stage_bytes;
   int cursor = 0;
 
   if (warp == kConsumerWarps) {
@@ -157,13 +160,13 @@ __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_co
         atomicAdd(&g_wait_timeouts_fold, 1u);
         break;
       }
-      const TileInfo ti = tile_info(tb, blockIdx.x + (uint64_t)k * Gd, cursor, a.tv);
-      unsigned char *st = smem + (size_t)s * a.stage_bytes;
+      const TileInfo ti = tile_info(tb, blockIdx.x + (uint64_t)k * Gd, cursor, tv);
+      unsigned char *st = smem + (size_t)s * stage_bytes;
       const uint32_t bytes = ti.nv * 16u;
       mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)p);
       const char *const *src = s_src[ti.seg];
       for (int q = 0; q < p; ++q)
-        bulk_load(st + (size_t)q * a.tile_bytes, src[q] + ti.v0 * 16, bytes, &full[s]);
+        bulk_load(st + (size_t)q * tile_bytes, src[q] + ti.v0 * 16, bytes, &full[s]);
       if (++s == S) {
         s = 0;
         ++use;
@@ -199,30 +202,44 @@ __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_co
       if (lane == 0) atomicAdd(&g_wait_timeouts_fold, 1u);
       break;
     }
-    const TileInfo ti = tile_info(tb, blockIdx.x + (uint64_t)k * Gd, cursor, a.tv);
-    const unsigned char *st = smem + (size_t)s * a.stage_bytes;
+    const TileInfo ti = tile_info(tb, blockIdx.x + (uint64_t)k * Gd, cursor, tv);
+    const uint32_t st = smem_addr(smem) + (uint32_t)s * stage_bytes;  // shared address
     char *d1 = (mode == kModeScatter) ? s_dst[tb.cg[ti.seg]] : dall[0];
     for (uint32_t v = ctid; v < ti.nv; v += kConsumerThreads) {
       Acc Sg[VEC], T[VEC];
+      const uint32_t col = st + v * 16u;
+      if constexpr (!GROUPED) {
+        unpack<TI>(lds128(col), T);
 #pragma unroll
-      for (int q = 0; q < PMAX; ++q) {
-        if (q < p) {
-          Acc x[VEC];
-          unpack<TI>(*reinterpret_cast<const uint4 *>(st + (size_t)q * a.tile_bytes + v * 16u), x);
-          if ((first >> q) & 1u) {
+        for (int q = 1; q < PMAX; ++q) {
+          if (q < p) {
+            Acc x[VEC];
+            unpack<TI>(lds128(col + (uint32_t)q * tile_bytes), x);
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) Sg[e] = x[e];
-          } else {
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) Sg[e] = combine<OP>(Sg[e], x[e]);
+            for (int e = 0; e < VEC; ++e) T[e] = combine<OP>(T[e], x[e]);
           }
-          if ((lastm >> q) & 1u) {
-            if (q < G) {
+        }
+      } else {
 #pragma unroll
-              for (int e = 0; e < VEC; ++e) T[e] = Sg[e];
+        for (int q = 0; q < PMAX; ++q) {
+          if (q < p) {
+            Acc x[VEC];
+            unpack<TI>(lds128(col + (uint32_t)q * tile_bytes), x);
+            if ((first >> q) & 1u) {
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) Sg[e] = x[e];
             } else {
 #pragma unroll
-              for (int e = 0; e < VEC; ++e) T[e] = combine<OP>(T[e], Sg[e]);
+              for (int e = 0; e < VEC; ++e) Sg[e] = combine<OP>(Sg[e], x[e]);
+            }
+            if ((lastm >> q) & 1u) {
+              if (q < G) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) T[e] = Sg[e];
+              } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) T[e] = combine<OP>(T[e], Sg[e]);
+              }
             }
           }
         }
@@ -306,15 +323,17 @@ cudaError_t run_fold(const FoldJob &job, cudaStream_t s) {
   a.stages = stages;
   const size_t smem = (size_t)stages * a.stage_bytes;
 
-  auto kern = rc_fold_tma_kernel<PMAX, TI, TO, OP>;
-  static std::atomic<uint64_t> attr_set{0};
+  auto kern = job.G == job.p ? rc_fold_tma_kernel<PMAX, TI, TO, OP, false>
+                             : rc_fold_tma_kernel<PMAX, TI, TO, OP, true>;
+  static std::atomic<uint64_t> attr_set[2];  // [GROUPED], one bit per device
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (!(attr_set.load() & (1ull << (dev & 63)))) {
+  std::atomic<uint64_t> &flag = attr_set[job.G == job.p ? 0 : 1];
+  if (!(flag.load() & (1ull << (dev & 63)))) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (err != cudaSuccess) return err;
-    attr_set.fetch_or(1ull << (dev & 63));
+    flag.fetch_or(1ull << (dev & 63));
   }
   int occ = 0;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kFoldNT, smem);

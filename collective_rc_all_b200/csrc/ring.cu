@@ -60,6 +60,16 @@ __device__ __forceinline__ uint4 ld_cg_v4(const void *p) {
                : "memory");
   return v;
 }
+// Default-cached (L1) loads: a thread's load after its own store to the same
+// address returns the stored value under either caching mode.
+__device__ __forceinline__ uint4 ld_ca_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.ca.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
 __device__ __forceinline__ uint32_t ld_cg_u32(const void *p) {
   uint32_t v;
   asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -109,7 +119,7 @@ __device__ __forceinline__ void unpack_raw(uint32_t raw, typename T::Acc (&a)[VE
 }
 
 // partial (raw 32-bit accumulators) load / store
-template <class Acc, int VEC>
+template <class Acc, int VEC, bool L1>
 __device__ __forceinline__ void load_part(const char *p, Acc (&a)[VEC]) {
   uint32_t w[VEC];
   if constexpr (VEC == 1) {
@@ -117,7 +127,7 @@ __device__ __forceinline__ void load_part(const char *p, Acc (&a)[VEC]) {
   } else {
 #pragma unroll
     for (int h = 0; h < VEC / 4; ++h) {
-      const uint4 v = ld_cg_v4(p + 16 * h);
+      const uint4 v = L1 ? ld_ca_v4(p + 16 * h) : ld_cg_v4(p + 16 * h);
       w[4 * h] = v.x;
       w[4 * h + 1] = v.y;
       w[4 * h + 2] = v.z;
@@ -174,7 +184,7 @@ struct AgEntry {      // all-gather step k, r -> d = r+1, chunk c = r-k
 // Registers are capped so that at least 4 (PMAX <= 8) or 2 (PMAX = 16) thread
 // blocks fit per SM: a typical launch then keeps every offset resident at
 // once, instead of running a second full 2(p-1)-step chain for a few blocks.
-template <class T, int OP, bool VECTOR, int PMAX>
+template <class T, int OP, bool VECTOR, int PMAX, bool L1>
 __global__ void __launch_bounds__(kRingNT, (PMAX <= 8 ? 4 : 2))
     rc_ring_literal_kernel(const __grid_constant__ RingParams a) {
   using Acc = typename T::Acc;
@@ -249,7 +259,7 @@ __global__ void __launch_bounds__(kRingNT, (PMAX <= 8 ? 4 : 2))
           const int r = r0 + g;
           if (r < p && oe < rs[k][r].len) {
             if (k == 0) unpack_raw<T, VEC>(load_raw<T, VEC>(rs[0][r].msg + oin), msg[g]);
-            else load_part<Acc, VEC>(rs[k][r].msg + o4, msg[g]);
+            else load_part<Acc, VEC, L1>(rs[k][r].msg + o4, msg[g]);
           }
         }
 #pragma unroll
@@ -284,7 +294,7 @@ __global__ void __launch_bounds__(kRingNT, (PMAX <= 8 ? 4 : 2))
       for (int r = 0; r < PMAX; ++r) {
         if (r < p && oe < ag[k][r].len) {
           const char *src = ag[k][r].src + oin;
-          if constexpr (VECTOR) v16[r] = ld_cg_v4(src);
+          if constexpr (VECTOR) v16[r] = L1 ? ld_ca_v4(src) : ld_cg_v4(src);
           else if constexpr (kIn == 2) v4[r] = ld_cg_u16(src);
           else v4[r] = ld_cg_u32(src);
         }
@@ -321,7 +331,10 @@ cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   constexpr int VEC = kVec<T>;
   const bool vector = aligned && a.C % VEC == 0 && a.n % VEC == 0;
   const int sms = device_sm_count();
-  auto kern = vector ? rc_ring_literal_kernel<T, OP, true, PMAX> : rc_ring_literal_kernel<T, OP, false, PMAX>;
+  const bool l1 = env_int("RC_RING_L1", 1) != 0;
+  auto kern = vector ? (l1 ? rc_ring_literal_kernel<T, OP, true, PMAX, true>
+                           : rc_ring_literal_kernel<T, OP, true, PMAX, false>)
+                     : rc_ring_literal_kernel<T, OP, false, PMAX, false>;
   a.units = vector ? a.C / VEC : a.C;
   int occ = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kRingNT, 0);
