@@ -23,7 +23,7 @@ __all__ = [
     "FP32", "BF16", "INT32", "SUM", "MAX", "MIN", "RING_LITERAL", "RING_ONESHOT",
     "HIER_FUSED", "HIER_STAGED",
     "rc_all_reduce", "rc_reduce_scatter", "rc_all_gather", "rc_reduce", "rc_broadcast",
-    "rc_ring_all_reduce", "rc_hier_all_reduce", "rc_copy", "rc_reserve_workspace", "rc_check_buffer",
+    "rc_ring_all_reduce", "rc_ring_all_reduce_noalloc", "rc_hier_all_reduce", "rc_copy", "rc_reserve_workspace", "rc_check_buffer",
     "rc_probe_bounded_wait",
     "rc_stream_status", "rc_launch_count", "rc_finalize", "rc_version", "rc_last_error",
 ]
@@ -63,6 +63,7 @@ _decl("rc_reduce", [_vpp, _vp, _i, _i, _sz, _i, _i, _f, _vp])
 _decl("rc_broadcast", [_vp, _vpp, _i, _i, _sz, _i, _vp])
 _decl("rc_ring_all_reduce", [_vpp, _vpp, _i, _sz, _i, _i, _f, _i, _vp])
 _decl("rc_hier_all_reduce", [_vpp, _vpp, _i, _i, _sz, _i, _i, _f, _i, _vp])
+_decl("rc_ring_all_reduce_noalloc", [_vpp, _vpp, _i, _sz, _i, _i, _f, _vp])
 _decl("rc_copy", [_vp, _vp, _sz, _vp])
 _decl("rc_reserve_workspace", [_sz, _vp])
 _decl("rc_check_buffer", [_vp, _sz])
@@ -195,6 +196,15 @@ def rc_ring_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], n=None, dtype=N
     _check(lib.rc_ring_all_reduce(_ptrs(send), _ptrs(recv), p, _numel(send[0], n),
                                   _dt(dtype, send[0]), _op(op), scale, int(v), _stream(stream)),
            "rc_ring_all_reduce")
+
+
+def rc_ring_all_reduce_noalloc(send: Sequence[Buf], recv: Sequence[Buf], n=None, dtype=None,
+                               op="sum", scale=1.0, stream=None):
+    """Literal ring all-reduce that allocates nothing (fixed scratch for bf16)."""
+    p = len(send)
+    _check(lib.rc_ring_all_reduce_noalloc(_ptrs(send), _ptrs(recv), p, _numel(send[0], n),
+                                          _dt(dtype, send[0]), _op(op), scale, _stream(stream)),
+           "rc_ring_all_reduce_noalloc")
 
 
 def rc_hier_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], group_size: int, n=None,

@@ -444,6 +444,44 @@ rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, 
   return st;
 }
 
+rc_status rc_ring_all_reduce_noalloc(const void *const *send, void *const *recv, int p, size_t n,
+                                     rc_dtype dt, rc_op op, float scale, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(dt, dt, op, scale)) != RC_OK) return st;
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  if (p == 1) return rc_all_reduce(send, recv, p, n, dt, op, scale, stream);  // no steps, no scratch
+  const uint64_t C = (n + p - 1) / p;
+  const uint64_t need = dt == RC_BF16 ? 2ull * p * C : 0;  // fp32 partials, bf16 only
+  if (need > noalloc_scratch_floats())
+    return fail(RC_ERR_INVALID_ARG,
+                "rc_ring_all_reduce_noalloc: bf16 with p=%d, n=%zu needs %llu floats of scratch; the "
+                "fixed scratch holds %zu (2*p*ceil(n/p) must not exceed it)",
+                p, n, (unsigned long long)need, noalloc_scratch_floats());
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, s, 0, r, false, "send", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  RingJob j{};
+  j.p = p;
+  j.n = n;
+  j.dt = dt;
+  j.op = op;
+  j.scale = scale;
+  for (int r = 0; r < p; ++r) {
+    j.x[r] = send[r];
+    j.y[r] = recv[r];
+  }
+  if (dt == RC_BF16) {
+    cudaError_t e = noalloc_scratch_ptr(&j.ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(fixed scratch)");
+  }
+  return launched(launch_ring_literal(j, (cudaStream_t)stream), "ring launch");
+}
+
 rc_status rc_hier_all_reduce(const void *const *send, void *const *recv, int p, int group_size,
                              size_t n, rc_dtype dt, rc_op op, float scale, rc_hier_variant variant,
                              rc_stream_t stream) {

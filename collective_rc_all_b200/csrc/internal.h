@@ -77,6 +77,8 @@ cudaError_t launch_fold_tma(const FoldJob &job, cudaStream_t s);
 cudaError_t read_and_clear_fold_timeouts(unsigned int *count);
 cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s);
 cudaError_t launch_ring_literal(const RingJob &job, cudaStream_t s);
+size_t noalloc_scratch_floats();
+cudaError_t noalloc_scratch_ptr(void **out);
 cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s);
 cudaError_t launch_hier_staged(const HierJob &job, cudaStream_t s);
 cudaError_t launch_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);

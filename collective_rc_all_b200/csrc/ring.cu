@@ -31,6 +31,7 @@
 // only the partials' round trip through L2 stays on the dependent chain.  The
 // per-(step, rank) chunk addresses come from a table in shared memory.
 #include <algorithm>
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -365,6 +366,38 @@ cudaError_t ring_by_op(const RingJob &job, cudaStream_t s) {
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for rc_ring_all_reduce_noalloc: the bf16 ring's fp32
+// partials, [2 parities][p][ceil(n/p)] floats, in a file-scope device array
+// instead of an allocation.  Every GPU that loads this library holds it until
+// the process exits.  Calls that use it and overlap on the GPU race on it.
+// Nothing in it needs clearing: every partial is written before it is read.
+constexpr size_t kNoallocScratchFloats = size_t(4) << 20;  // 16 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchFloats];
+
+size_t noalloc_scratch_floats() { return kNoallocScratchFloats; }
+
+// Device address of the array for the current device.  In host code the
+// symbol's name is only a host-side handle, so the address is looked up once
+// per device (with that device current) and cached.
+cudaError_t noalloc_scratch_ptr(void **out) {
+  static std::mutex mu;
+  static void *ptrs[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess) return err;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
 
 cudaError_t launch_ring_literal(const RingJob &job, cudaStream_t s) {
   switch (job.dt) {

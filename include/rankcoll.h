@@ -153,6 +153,33 @@ rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, 
                              rc_stream_t stream);
 
 /*
+ * ring all-reduce that allocates nothing.  The pages have no counterpart of
+ * this entry point; it exists for callers that cannot allocate device memory
+ * at call time: code whose device memory is owned entirely by another
+ * allocator (a framework's caching allocator that must remain the only one),
+ * code that must not stall on cudaMalloc/cudaFree (both can synchronise the
+ * device), and code running where allocation is not allowed.
+ *
+ * Same arguments, result bits and literal schedule as rc_ring_all_reduce with
+ * RC_RING_LITERAL.  For bf16 the fp32 partials live in a fixed scratch array
+ * inside this library (16 MiB of device memory, held by every GPU that loads
+ * the library until the process exits) instead of the library workspace, so
+ * bf16 calls need 2 * p * ceil(n/p) <= 4,194,304; larger requests return
+ * RC_ERR_INVALID_ARG with the limit in rc_last_error.  fp32 and int32 keep
+ * their partials in recv and use no scratch.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (once per device, that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    calls whose kernels overlap on the GPU (for example on two streams) race
+ *    on it.  Nothing in it needs clearing: every partial is written before it
+ *    is read.
+ *  - Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+rc_status rc_ring_all_reduce_noalloc(const void *const *send, void *const *recv, int p, size_t n,
+                                     rc_dtype dt, rc_op op, float scale, rc_stream_t stream);
+
+/*
  * hierarchical all-reduce [HIER]: ranks form p/group_size contiguous groups
  * of group_size.  (1) each group's ranks are folded in ring order over the
  * group (chunk length ceil(n/group_size)); (2) the groups' results are folded
