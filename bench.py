@@ -461,6 +461,108 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------------------ sweep workload
+def run_sweep(args):
+    """The sweep configuration: p in {2,4,8,16}, per-rank sizes 1 KiB .. max in
+    powers of 4, fp32/bf16/int32, all_reduce and reduce_scatter with sum and
+    max, all_gather.  One JSON line per point: single-call device time (L2
+    flushed before every call, outside the events), effective GB/s on the
+    minimum-bytes basis, and for sizes <= 4 MiB the per-call time inside a
+    CUDA graph of 20 back-to-back calls (the launch-latency term)."""
+    import torch
+    import collective_rc_all_b200 as rc
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    peak, _ = measured_peaks()
+    TT = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}
+    ESZ = {"f32": 4, "bf16": 2, "i32": 4}
+    gen = torch.Generator(device=dev)
+    sizes = [1 << k for k in range(10, 31, 2) if (1 << k) <= args.sweep_max_bytes]
+    out = open(args.sweep_out, "w") if args.sweep_out else None
+
+    def time_call(fn, footprint, reps):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            # always flush (untimed): without it the previous call's dirty
+            # outputs are written back inside the timed call
+            flush.zero_()
+            torch.sum(clean, dim=0, out=sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e-3)
+        return float(np.median(ts)), float(min(ts))
+
+    def time_graph(fn, calls=20):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for _ in range(calls):
+                fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e-3 / calls)
+        del g
+        return float(np.median(ts))
+
+    for p in (2, 4, 8, 16):
+        for nbytes in sizes:
+            for dt in ("f32", "bf16", "i32"):
+                s = ESZ[dt]
+                n = nbytes // s
+                gen.manual_seed(100 + p * 131 + nbytes % 10007)
+                if dt == "i32":
+                    send = [torch.randint(-(1 << 20), 1 << 20, (n,), generator=gen, device=dev,
+                                          dtype=torch.int32) for _ in range(p)]
+                else:
+                    send = [(torch.rand(n, generator=gen, device=dev) * 2 - 1).to(TT[dt]) for _ in range(p)]
+                y = [torch.empty(n, dtype=TT[dt], device=dev) for _ in range(p)]
+                rs = [torch.empty(n // p, dtype=TT[dt], device=dev) for _ in range(p)]
+                cases = [
+                    ("all_reduce", "sum", lambda: rc.rc_all_reduce(send, y, op="sum"), 2 * p * n * s),
+                    ("all_reduce", "max", lambda: rc.rc_all_reduce(send, y, op="max"), 2 * p * n * s),
+                    ("reduce_scatter", "sum", lambda: rc.rc_reduce_scatter(send, rs, op="sum"), p * n * s + n * s),
+                    ("reduce_scatter", "max", lambda: rc.rc_reduce_scatter(send, rs, op="max"), p * n * s + n * s),
+                    ("all_gather", "-", lambda: rc.rc_all_gather(rs, y), n * s + p * n * s),
+                ]
+                reps = 20 if nbytes <= (64 << 20) else 5
+                for coll, op, fn, byt in cases:
+                    med, mn = time_call(fn, byt, reps)
+                    row = {"p": p, "bytes_per_rank": nbytes, "dtype": dt, "coll": coll, "op": op,
+                           "us": round(med * 1e6, 2), "us_min": round(mn * 1e6, 2),
+                           "gbs": round(byt / med / 1e9, 1), "frac_of_measured_hbm": round(byt / med / 1e9 / peak, 4)}
+                    if nbytes <= (4 << 20):
+                        tg = time_graph(fn)
+                        row["us_in_graph"] = round(tg * 1e6, 2)
+                        row["gbs_in_graph"] = round(byt / tg / 1e9, 1)
+                    line = json.dumps(row)
+                    print(line, flush=True)
+                    if out:
+                        out.write(line + "\n")
+                del send, y, rs
+                torch.cuda.empty_cache()
+    rc.rc_stream_status()
+    if out:
+        out.close()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -475,10 +577,16 @@ def main(argv=None):
     ap.add_argument("--ops", default="", help="comma-separated subset of the step's collectives")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-copy-peak", action="store_true")
+    # the sweep workload (not the driver's step): one JSON line per point
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--sweep-max-bytes", type=int, default=1 << 30)
+    ap.add_argument("--sweep-out", default="")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 
