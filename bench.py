@@ -136,7 +136,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -340,14 +340,16 @@ def run_ours(args):
         copy_gbs = 2 * (1 << 30) / min(cps) / 1e9
         del cp_a, cp_b
 
+    # the clock sampler starts before the warm-up, so the GPU is busy (not
+    # idling at low clocks) when the timed region begins
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
     for _ in range(W):
         one_step()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    time.sleep(0.3)
     torch.cuda.synchronize()
     launches0 = rc.rc_launch_count()
     for k in range(K):
@@ -361,6 +363,7 @@ def run_ours(args):
     rc.rc_stream_status()
 
     per_op_s = {nm: sum(a.elapsed_time(b) for a, b in ev[nm]) * 1e-3 for nm in names}
+    per_op_dist = {nm: sorted(a.elapsed_time(b) * 1e-3 for a, b in ev[nm]) for nm in names}
     local_s = sum(per_op_s.values())
     tot_s, tot_bytes = reduce_over_ranks(local_s, step_bytes * K, world, device=dev)
 
@@ -411,7 +414,10 @@ def run_ours(args):
     per_op = {}
     for nm, b in ops:
         t = per_op_s[nm] / K
-        per_op[nm] = {"us": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
+        dist = per_op_dist[nm]
+        per_op[nm] = {"us": round(t * 1e6, 2), "us_median": round(dist[len(dist) // 2] * 1e6, 2),
+                      "us_min": round(dist[0] * 1e6, 2), "us_max": round(dist[-1] * 1e6, 2),
+                      "gbs": round(b / t / 1e9, 1),
                       "frac_of_measured_hbm": round(b / t / 1e9 / peak, 4),
                       "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4) if copy_gbs else None}
     if "all_reduce" in per_op:
