@@ -58,7 +58,14 @@ WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 
 # DRAM traffic per launch measured by ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum) for the kernel named, together with a hash of the
 # kernel's source file when it was measured; a changed source reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # op: DRAM bytes per launch (read + write, one cold-cache ncu launch of the
+    # step's workload), kernel source hash at capture time
+    "ring_all_reduce": {"bytes": 68177408 + 51077376, "src": "4d84d550ed796b2e"},
+    "all_reduce": {"bytes": 67133440 + 22459392, "src": "db7c2d49405fa2d0"},
+    "reduce_scatter": {"bytes": 67121408 + 987904, "src": "1a713eca9a1f13ac"},
+    "all_gather": {"bytes": 4205312 + 726528, "src": "216eaf2ee5963ca6"},
+}
 
 
 def busbw_all_reduce(size_bytes: float, p: int, t: float) -> float:
@@ -95,13 +102,13 @@ def step_ops(p=P, n=N):
 
 
 KERNEL_OF = {
-    "all_reduce": ("reduce_kernel", "reduce.cu"),
-    "reduce_scatter": ("reduce_kernel", "reduce.cu"),
-    "all_gather": ("fanout_bulk_kernel", "fanout.cu"),
-    "reduce": ("reduce_kernel", "reduce.cu"),
-    "broadcast": ("fanout_bulk_kernel", "fanout.cu"),
-    "ring_all_reduce": ("ring_literal_kernel", "ring.cu"),
-    "hier_all_reduce": ("hier_fused_kernel", "hier.cu"),
+    "all_reduce": ("rc_fold_tma_kernel", "fold.cu"),
+    "reduce_scatter": ("rc_reduce_front_kernel", "reduce.cu"),
+    "all_gather": ("rc_fanout_bulk_kernel", "fanout.cu"),
+    "reduce": ("rc_reduce_front_kernel", "reduce.cu"),
+    "broadcast": ("rc_fanout_bulk_kernel", "fanout.cu"),
+    "ring_all_reduce": ("rc_ring_literal_kernel", "ring.cu"),
+    "hier_all_reduce": ("rc_fold_tma_kernel", "fold.cu"),
 }
 
 
@@ -415,7 +422,10 @@ def run_ours(args):
     for nm, b in ops:
         t = per_op_s[nm] / K
         dist = per_op_dist[nm]
+        trf = NCU_TRAFFIC.get(nm)
+        per_op_traffic = trf["bytes"] if trf and trf["src"] == _src_hash(KERNEL_OF[nm][1]) else None
         per_op[nm] = {"us": round(t * 1e6, 2), "us_median": round(dist[len(dist) // 2] * 1e6, 2),
+                      "ncu_dram_bytes": per_op_traffic, "algorithmic_bytes": b,
                       "us_min": round(dist[0] * 1e6, 2), "us_max": round(dist[-1] * 1e6, 2),
                       "gbs": round(b / t / 1e9, 1),
                       "frac_of_measured_hbm": round(b / t / 1e9 / peak, 4),
