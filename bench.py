@@ -8,11 +8,16 @@ seed 1 (the ring / one-shot all-reduce workload), through
   all_reduce (one-shot), reduce_scatter (fp32 -> bf16, scale 1/8),
   all_gather (the bf16 shards), reduce (root 0), broadcast (root 0, in place),
   ring all_reduce (literal 14 steps), hierarchical all_reduce (2 x 4, fused).
-Each collective is timed alone with CUDA events on the launching stream.  An
-L2 flush runs between collectives, outside the timed events: a 512 MiB write
-(more than the 126 MB L2) followed by a 256 MiB read of another buffer, so
-every collective reads its inputs from HBM and starts with an L2 that holds
-no dirty lines of someone else's (the flush's) data to write back.
+Timing: each collective is captured once into a CUDA graph; the K steps
+replay the graphs back to back between one pair of CUDA events on the
+launching stream (an event between consecutive collectives splits the time
+per collective).  Every collective of the step has its own inputs and outputs,
+so between two reads of an op's inputs the other six move more than 500 MiB
+(over 4x the 126 MB L2): the inputs come from HBM ("inputs larger than L2").
+A second view times every collective alone after an L2 flush outside its
+events (a 512 MiB write, then a 256 MiB read of another buffer, so L2 holds no
+dirty lines of the flush's to write back).  CUDA event timestamps here tick
+at about 2 us, so per-collective figures are means over many steps.
 
 Effective GB/s = minimum bytes read + written / device time (decimal GB):
   all_reduce p*n*s_in + p*n*s_out; reduce_scatter p*n*s_in + n*s_out;
@@ -279,15 +284,21 @@ def run_ours(args):
     ops, m = step_ops()
     step_bytes = sum(b for _, b in ops)
 
-    # inputs: each replica draws its own batch (seed + rank)
+    # inputs: each replica draws its own batch (seed + rank); every collective
+    # of the step gets its own copy of the inputs and its own outputs, so in
+    # the back-to-back timing the inputs an op reads were last touched a whole
+    # step (> 500 MiB of traffic, > 4x L2) earlier and come from HBM
     xs = rc_inputs.normal(P, N, seed=SEED + rank, sigma=SIGMA)
     send = [torch.from_numpy(x).to(dev) for x in xs]
+    own = lambda: [t.clone() for t in send]
     f32 = lambda k: [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(k)]
+    bf16 = lambda k, n: [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(k)]
+    s_ar, s_rs, s_red, s_bc, s_ring, s_hier = own(), own(), own(), own(), own(), own()
     y_ar, y_ring, y_hier = f32(P), f32(P), f32(P)
-    y_rs = [torch.empty(m, dtype=torch.bfloat16, device=dev) for _ in range(P)]
-    y_ag = [torch.empty(N, dtype=torch.bfloat16, device=dev) for _ in range(P)]
+    y_rs, ag_in, y_ag = bf16(P, m), bf16(P, m), bf16(P, N)
     y_red = torch.empty(N, dtype=torch.float32, device=dev)
-    y_bc = [send[0]] + f32(P - 1)          # root 0 in place
+    y_bc = [s_bc[0]] + f32(P - 1)          # root 0 in place
+    rc.rc_reduce_scatter(send, ag_in, out_dtype="bf16", scale=1.0 / P)  # the all-gather's shards
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -297,13 +308,13 @@ def run_ours(args):
         torch.sum(clean, dim=0, out=sink)
 
     calls = {
-        "all_reduce": lambda: rc.rc_all_reduce(send, y_ar),
-        "reduce_scatter": lambda: rc.rc_reduce_scatter(send, y_rs, out_dtype="bf16", scale=1.0 / P),
-        "all_gather": lambda: rc.rc_all_gather(y_rs, y_ag),
-        "reduce": lambda: rc.rc_reduce(send, y_red, root=0),
-        "broadcast": lambda: rc.rc_broadcast(send[0], y_bc, root=0),
-        "ring_all_reduce": lambda: rc.rc_ring_all_reduce(send, y_ring, variant="literal"),
-        "hier_all_reduce": lambda: rc.rc_hier_all_reduce(send, y_hier, 4, variant="fused"),
+        "all_reduce": lambda: rc.rc_all_reduce(s_ar, y_ar),
+        "reduce_scatter": lambda: rc.rc_reduce_scatter(s_rs, y_rs, out_dtype="bf16", scale=1.0 / P),
+        "all_gather": lambda: rc.rc_all_gather(ag_in, y_ag),
+        "reduce": lambda: rc.rc_reduce(s_red, y_red, root=0),
+        "broadcast": lambda: rc.rc_broadcast(s_bc[0], y_bc, root=0),
+        "ring_all_reduce": lambda: rc.rc_ring_all_reduce(s_ring, y_ring, variant="literal"),
+        "hier_all_reduce": lambda: rc.rc_hier_all_reduce(s_hier, y_hier, 4, variant="fused"),
     }
     if args.ops:
         keep = args.ops.split(",")
@@ -314,19 +325,29 @@ def run_ours(args):
         step_bytes = sum(b for _, b in ops)
     names = [nm for nm, _ in ops]
     K, W = args.steps, args.warmup
-    ev = {nm: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)] for nm in names}
+    # back-to-back timing: every collective is captured once into its own CUDA
+    # graph (one host launch per collective instead of the binding's argument
+    # marshalling and checks, which take longer than a collective on the GPU);
+    # one event before every collective of every step and one after the last
+    for nm in names:
+        calls[nm]()  # first calls outside capture (one-time set-up)
+    torch.cuda.synchronize()
+    graphs, launches_per_graph = {}, {}
+    for nm in names:
+        g = torch.cuda.CUDAGraph()
+        l0 = rc.rc_launch_count()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            calls[nm]()
+        launches_per_graph[nm] = rc.rc_launch_count() - l0
+        graphs[nm] = g
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K * len(names) + 1)]
 
     def one_step(k=None):
-        for nm in names:
-            l2_flush()                          # untimed: evicts L2 before each collective
-            if k is None:
-                calls[nm]()
-            else:
-                a, b = ev[nm][k]
-                a.record(stream)
-                calls[nm]()
-                b.record(stream)
+        for j, nm in enumerate(names):
+            if k is not None:
+                evs[k * len(names) + j].record(stream)
+            graphs[nm].replay()
 
     # copy roofline of this library's own copy kernel (same run), 1 GiB
     copy_gbs = None
@@ -358,20 +379,44 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    launches0 = rc.rc_launch_count()
     for k in range(K):
         one_step(k)
+    evs[-1].record(stream)
     torch.cuda.synchronize()
-    launches = rc.rc_launch_count() - launches0
+    # this library's kernels inside the timed region: the kernels each
+    # captured graph holds, times its replays
+    launches = K * sum(launches_per_graph.values())
     time.sleep(0.3)
     clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
     rc.rc_stream_status()
 
-    per_op_s = {nm: sum(a.elapsed_time(b) for a, b in ev[nm]) * 1e-3 for nm in names}
-    per_op_dist = {nm: sorted(a.elapsed_time(b) * 1e-3 for a, b in ev[nm]) for nm in names}
-    local_s = sum(per_op_s.values())
+    # second view: every collective alone, L2 flushed (untimed) before it
+    iso_k = min(K, 30)
+    iso = {nm: [] for nm in names}
+    for _ in range(iso_k):
+        for nm in names:
+            l2_flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            calls[nm]()
+            b.record(stream)
+            b.synchronize()
+            iso[nm].append(a.elapsed_time(b) * 1e-3)
+    rc.rc_stream_status()
+
+    total_s = evs[0].elapsed_time(evs[-1]) * 1e-3
+    per_op_s = {nm: 0.0 for nm in names}
+    per_op_all = {nm: [] for nm in names}
+    for k in range(K):
+        for j, nm in enumerate(names):
+            i = k * len(names) + j
+            dt_ = evs[i].elapsed_time(evs[i + 1]) * 1e-3
+            per_op_s[nm] += dt_
+            per_op_all[nm].append(dt_)
+    per_op_dist = {nm: sorted(v) for nm, v in per_op_all.items()}
+    local_s = total_s
     tot_s, tot_bytes = reduce_over_ranks(local_s, step_bytes * K, world, device=dev)
 
     # ---- end to end through the same calls with host buffers (pinned)
@@ -385,11 +430,23 @@ def run_ours(args):
     if args.no_e2e:
         e2e_k = 0
 
+    # end to end: one set of inputs copied in from the host, every collective
+    # of the step on it, one copy of every result copied back
+    e2e_calls = {
+        "all_reduce": lambda: rc.rc_all_reduce(send, y_ar),
+        "reduce_scatter": lambda: rc.rc_reduce_scatter(send, y_rs, out_dtype="bf16", scale=1.0 / P),
+        "all_gather": lambda: rc.rc_all_gather(y_rs, y_ag),
+        "reduce": lambda: rc.rc_reduce(send, y_red, root=0),
+        "broadcast": lambda: rc.rc_broadcast(send[0], [send[0]] + y_bc[1:], root=0),
+        "ring_all_reduce": lambda: rc.rc_ring_all_reduce(send, y_ring, variant="literal"),
+        "hier_all_reduce": lambda: rc.rc_hier_all_reduce(send, y_hier, 4, variant="fused"),
+    }
+
     def e2e_step():
         for d, h in zip(send, host_in):
             d.copy_(h, non_blocking=True)
         for nm in names:
-            calls[nm]()
+            e2e_calls[nm]()
         for h, d in zip(host_out, flat_outs):
             h.copy_(d, non_blocking=True)
 
@@ -422,14 +479,16 @@ def run_ours(args):
     for nm, b in ops:
         t = per_op_s[nm] / K
         dist = per_op_dist[nm]
+        ti = float(np.mean(iso[nm]))
         trf = NCU_TRAFFIC.get(nm)
         per_op_traffic = trf["bytes"] if trf and trf["src"] == _src_hash(KERNEL_OF[nm][1]) else None
         per_op[nm] = {"us": round(t * 1e6, 2), "us_median": round(dist[len(dist) // 2] * 1e6, 2),
                       "ncu_dram_bytes": per_op_traffic, "algorithmic_bytes": b,
-                      "us_min": round(dist[0] * 1e6, 2), "us_max": round(dist[-1] * 1e6, 2),
                       "gbs": round(b / t / 1e9, 1),
                       "frac_of_measured_hbm": round(b / t / 1e9 / peak, 4),
-                      "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4) if copy_gbs else None}
+                      "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4) if copy_gbs else None,
+                      "isolated_us": round(ti * 1e6, 2),
+                      "isolated_frac_of_measured_hbm": round(b / ti / 1e9 / peak, 4)}
     if "all_reduce" in per_op:
         t_ar = per_op_s["all_reduce"] / K
         per_op["all_reduce"]["busbw_gib_s"] = round(busbw_all_reduce(N * 4, P, t_ar) / 2**30, 1)
@@ -459,7 +518,12 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "p": P, "n_per_rank": N,
-                   "l2": "flushed (512 MiB write) before every collective, outside the timed events",
+                   "l2": ("inputs larger than L2: each collective of the step has its own inputs and "
+                          "outputs, so between two reads of an op's inputs the other ops move > 500 MiB "
+                          "(> 4x the 126 MB L2); the K steps replay one CUDA graph per collective back "
+                          "to back between one pair of CUDA events. per_op.isolated_*: each collective "
+                          "alone (plain call) after a 512 MiB write + "
+                          "256 MiB read L2 flush outside its events"),
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": kname, "op": dom,
                      "achieved": round(dom_b / dom_t / 1e9, 1), "peak": peak,
