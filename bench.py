@@ -8,10 +8,13 @@ seed 1 (the ring / one-shot all-reduce workload), through
   all_reduce (one-shot), reduce_scatter (fp32 -> bf16, scale 1/8),
   all_gather (the bf16 shards), reduce (root 0), broadcast (root 0, in place),
   ring all_reduce (literal 14 steps), hierarchical all_reduce (2 x 4, fused).
-Timing: each collective is captured once into a CUDA graph; the K steps
-replay the graphs back to back between one pair of CUDA events on the
-launching stream (an event between consecutive collectives splits the time
-per collective).  Every collective of the step has its own inputs and outputs,
+Timing: the whole step is captured once into a CUDA graph and the K steps
+replay it between one pair of CUDA events on the launching stream (the
+library launches its kernels with programmatic dependent launch, so inside
+the graph each kernel's launch overlaps the previous kernel's tail).  A split
+per collective replays one graph per collective K more times, with an event
+between consecutive collectives (`--graph per_op` makes that the headline).
+Every collective of the step has its own inputs and outputs,
 so between two reads of an op's inputs the other six move more than 500 MiB
 (over 4x the 126 MB L2): the inputs come from HBM ("inputs larger than L2").
 A second view times every collective alone after an L2 flush outside its
@@ -327,8 +330,14 @@ def run_ours(args):
     K, W = args.steps, args.warmup
     # back-to-back timing: every collective is captured once into its own CUDA
     # graph (one host launch per collective instead of the binding's argument
-    # marshalling and checks, which take longer than a collective on the GPU);
-    # one event before every collective of every step and one after the last
+    # marshalling and checks, which take longer than a collective on the GPU),
+    # and the whole step once more into one graph.  The headline replays the
+    # step graph K times between one pair of events: inside it, every kernel
+    # is launched with programmatic dependent launch, so its launch and
+    # prologue overlap the previous kernel's tail (each kernel still waits for
+    # the previous one to finish before it touches memory).  The split per
+    # collective replays the per-collective graphs K times with an event
+    # before every collective and one after the last.
     for nm in names:
         calls[nm]()  # first calls outside capture (one-time set-up)
     torch.cuda.synchronize()
@@ -340,6 +349,16 @@ def run_ours(args):
             calls[nm]()
         launches_per_graph[nm] = rc.rc_launch_count() - l0
         graphs[nm] = g
+    step_graph = None
+    if args.graph == "step":
+        step_graph = torch.cuda.CUDAGraph()
+        l0 = rc.rc_launch_count()
+        with torch.cuda.graph(step_graph, capture_error_mode="thread_local"):
+            for nm in names:
+                calls[nm]()
+        launches_per_step = rc.rc_launch_count() - l0
+    else:
+        launches_per_step = sum(launches_per_graph.values())
     torch.cuda.synchronize()
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K * len(names) + 1)]
 
@@ -374,18 +393,34 @@ def run_ours(args):
     clocks.start()
     time.sleep(0.3)
     for _ in range(W):
-        one_step()
+        if step_graph is not None:
+            step_graph.replay()
+        else:
+            one_step()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    if step_graph is not None:
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        for _ in range(K):
+            step_graph.replay()
+        eb.record(stream)
+        torch.cuda.synchronize()
+        step_s = ea.elapsed_time(eb) * 1e-3
+        if world > 1:
+            torch.distributed.barrier()
+    # the split per collective (the headline too when --graph per_op)
     for k in range(K):
         one_step(k)
     evs[-1].record(stream)
     torch.cuda.synchronize()
-    # this library's kernels inside the timed region: the kernels each
-    # captured graph holds, times its replays
-    launches = K * sum(launches_per_graph.values())
+    if step_graph is None:
+        step_s = evs[0].elapsed_time(evs[-1]) * 1e-3
+    # this library's kernels inside the headline's timed region: the kernels
+    # the captured graph(s) hold, times the replays
+    launches = K * launches_per_step
     time.sleep(0.3)
     clk = clocks.stop()
     if world > 1:
@@ -406,7 +441,7 @@ def run_ours(args):
             iso[nm].append(a.elapsed_time(b) * 1e-3)
     rc.rc_stream_status()
 
-    total_s = evs[0].elapsed_time(evs[-1]) * 1e-3
+    split_s = evs[0].elapsed_time(evs[-1]) * 1e-3
     per_op_s = {nm: 0.0 for nm in names}
     per_op_all = {nm: [] for nm in names}
     for k in range(K):
@@ -416,7 +451,7 @@ def run_ours(args):
             per_op_s[nm] += dt_
             per_op_all[nm].append(dt_)
     per_op_dist = {nm: sorted(v) for nm, v in per_op_all.items()}
-    local_s = total_s
+    local_s = step_s
     tot_s, tot_bytes = reduce_over_ranks(local_s, step_bytes * K, world, device=dev)
 
     # ---- end to end through the same calls with host buffers (pinned)
@@ -520,16 +555,22 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "p": P, "n_per_rank": N,
                    "l2": ("inputs larger than L2: each collective of the step has its own inputs and "
                           "outputs, so between two reads of an op's inputs the other ops move > 500 MiB "
-                          "(> 4x the 126 MB L2); the K steps replay one CUDA graph per collective back "
-                          "to back between one pair of CUDA events. per_op.isolated_*: each collective "
-                          "alone (plain call) after a 512 MiB write + "
-                          "256 MiB read L2 flush outside its events"),
+                          "(> 4x the 126 MB L2). " + (
+                              "value: K replays of one CUDA graph of the whole step between one pair of "
+                              "CUDA events (kernels with programmatic dependent launch); per_op.us: K "
+                              "replays of one graph per collective, back to back, an event between "
+                              "collectives" if step_graph is not None else
+                              "value and per_op.us: K replays of one CUDA graph per collective, back to "
+                              "back, an event between collectives") +
+                          ". per_op.isolated_*: each collective alone (plain call) after a 512 MiB "
+                          "write + 256 MiB read L2 flush outside its events"),
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": kname, "op": dom,
                      "achieved": round(dom_b / dom_t / 1e9, 1), "peak": peak,
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                      "unit": "GB/s", "frac": round(dom_b / dom_t / 1e9 / peak, 4),
                      "traffic": traffic, "algorithmic_bytes": dom_b},
+        "split_ms_per_step": round(1e3 * split_s / K, 4),
         "per_op": per_op,
         "copy_kernel_gbs": round(copy_gbs, 1) if copy_gbs else None,
         "cpu_baseline": cpu,
@@ -657,6 +698,8 @@ def main(argv=None):
     ap.add_argument("--ops", default="", help="comma-separated subset of the step's collectives")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-copy-peak", action="store_true")
+    ap.add_argument("--graph", choices=["step", "per_op"], default="step",
+                    help="headline from one CUDA graph of the whole step, or from one graph per collective")
     # the sweep workload (not the driver's step): one JSON line per point
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--sweep-max-bytes", type=int, default=1 << 30)

@@ -55,6 +55,11 @@ int device_sm_count() {
   return v;
 }
 
+bool pdl_enabled() {
+  static const bool on = env_int("RC_PDL", 1) != 0;
+  return on;
+}
+
 void note_launches(int k) { g_launches.fetch_add((uint64_t)k, std::memory_order_relaxed); }
 
 int env_int(const char *name, int dflt) {

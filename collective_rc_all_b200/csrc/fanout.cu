@@ -23,6 +23,7 @@
 #include "bulk.cuh"
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace rc {
 
@@ -56,6 +57,8 @@ __global__ void __launch_bounds__(32) rc_fanout_bulk_kernel(const __grid_constan
 
   for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
   mbar_init_fence();
+  pdl_wait();
+  pdl_trigger();
 
   const uint64_t G = gridDim.x;
   const uint64_t u0 = a.units * blockIdx.x / G;
@@ -116,6 +119,8 @@ __global__ void __launch_bounds__(32) rc_fanout_bulk_kernel(const __grid_constan
 // of 16 bytes): element copies, blockIdx.y = destination rank, x grid-stride.
 template <typename E>
 __global__ void rc_fanout_elem_kernel(const __grid_constant__ FanoutParams a, int nsrc) {
+  pdl_wait();
+  pdl_trigger();
   const int q = blockIdx.y;
   const uint64_t per_src = a.src_bytes / sizeof(E);
   const uint64_t total = per_src * nsrc;
@@ -192,18 +197,16 @@ cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s) {
       return err;
     occ = std::max(1, std::min(occ, env_int("RC_FANOUT_CTAS_PER_SM", 8)));
     const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>((uint64_t)sms * occ, a.units));
-    rc_fanout_bulk_kernel<<<(unsigned)grid, 32, smem, s>>>(a);
+    return launch_kernel(rc_fanout_bulk_kernel, dim3((unsigned)grid), dim3(32), smem, s, a);
   } else {
     const uint64_t per_src = job.src_bytes / job.elem_bytes;
     const uint64_t total = per_src * job.nsrc;
     const unsigned gx = (unsigned)std::max<uint64_t>(
         1, std::min<uint64_t>((total + 255) / 256, (uint64_t)sms * 4));
     dim3 grid(gx, job.p);
-    if (job.elem_bytes == 2) rc_fanout_elem_kernel<uint16_t><<<grid, 256, 0, s>>>(a, job.nsrc);
-    else rc_fanout_elem_kernel<uint32_t><<<grid, 256, 0, s>>>(a, job.nsrc);
+    if (job.elem_bytes == 2) return launch_kernel(rc_fanout_elem_kernel<uint16_t>, grid, dim3(256), 0, s, a, job.nsrc);
+    return launch_kernel(rc_fanout_elem_kernel<uint32_t>, grid, dim3(256), 0, s, a, job.nsrc);
   }
-  note_launches(1);
-  return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_wait_timeouts(unsigned int *count) {

@@ -38,6 +38,7 @@
 #include "bulk.cuh"
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace rc {
 
@@ -143,6 +144,8 @@ __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_co
     mbar_init_fence();
   }
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
 
   const uint64_t Gd = gridDim.x;
   const int64_t K = a.ntiles > blockIdx.x ? (int64_t)((a.ntiles - blockIdx.x + Gd - 1) / Gd) : 0;
@@ -340,9 +343,7 @@ cudaError_t run_fold(const FoldJob &job, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   occ = std::max(1, std::min(occ, env_int("RC_FOLD_CTAS", occ)));
   const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>((uint64_t)device_sm_count() * occ, tiles));
-  kern<<<(unsigned)grid, kFoldNT, smem, s>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kFoldNT), smem, s, a);
 }
 
 template <class TI, class TO, int OP>

@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace rc {
 namespace {
@@ -43,6 +44,8 @@ __global__ void __launch_bounds__(kNT) rc_hier_reg_kernel(const __grid_constant_
   using Acc = typename T::Acc;
   constexpr int VEC = VECTOR ? kVec<T> : 1;
   const int p = a.p, G = a.G, ng = a.ng;
+  pdl_wait();
+  pdl_trigger();
   const uint64_t Gd = gridDim.x;
   uint64_t u0 = a.units * blockIdx.x / Gd;
   const uint64_t u1 = a.units * (blockIdx.x + 1) / Gd;
@@ -139,9 +142,7 @@ cudaError_t run_fused(const HierJob &job, cudaStream_t s) {
   occ = std::max(1, std::min(occ, env_int("RC_CTAS_PER_SM", occ)));
   uint64_t grid = std::min<uint64_t>((uint64_t)device_sm_count() * occ, (a.units + kNT - 1) / kNT);
   grid = std::max<uint64_t>(grid, 1);
-  kern<<<(unsigned)grid, kNT, 0, s>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kNT), 0, s, a);
 }
 
 template <class T, int OP>

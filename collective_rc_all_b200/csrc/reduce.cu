@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace rc {
 namespace {
@@ -57,6 +58,8 @@ __device__ __forceinline__ int rot(uint64_t c, int k, int p) {
 template <int PMAX, class TI, class TO, int OP>
 __global__ void __launch_bounds__(kNT) rc_reduce_scalar_kernel(const __grid_constant__ ReduceParams a) {
   using Acc = typename TI::Acc;
+  pdl_wait();
+  pdl_trigger();
   const int p = a.p;
   const uint64_t G = gridDim.x;
   uint64_t u0 = a.nvec * blockIdx.x / G;
@@ -93,6 +96,8 @@ template <int PMAX, class TI, class TO, int OP, int ILP>
 __global__ void __launch_bounds__(kNT) rc_reduce_front_kernel(const __grid_constant__ ReduceParams a,
                                                               uint64_t tiles_per_chunk) {
   using Acc = typename TI::Acc;
+  pdl_wait();
+  pdl_trigger();
   constexpr int VEC = kVec<TI>;
   const int p = a.p;
   const uint64_t cvec = a.C / VEC;
@@ -151,6 +156,8 @@ template <int PMAX, class TI, class TO, int OP>
 __global__ void __launch_bounds__(32) rc_reduce_tail_kernel(const __grid_constant__ ReduceParams a,
                                                           uint64_t first) {
   using Acc = typename TI::Acc;
+  pdl_wait();
+  pdl_trigger();
   const int p = a.p;
   for (uint64_t e = first + threadIdx.x; e < a.n; e += blockDim.x) {
     const uint64_t c = e / a.C;
@@ -213,9 +220,9 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
     if ((err = launch_fold_tma(f, s)) != cudaSuccess) return err;
     a.nvec = n / VEC;
     if (a.nvec * VEC < n) {
-      rc_reduce_tail_kernel<PMAX, TI, TO, OP><<<1, 32, 0, s>>>(a, a.nvec * VEC);
-      note_launches(1);
-      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+      if ((err = launch_kernel(rc_reduce_tail_kernel<PMAX, TI, TO, OP>, dim3(1), dim3(32), 0, s, a,
+                               a.nvec * VEC)) != cudaSuccess)
+        return err;
     }
     return cudaSuccess;
   }
@@ -227,14 +234,14 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
       const uint64_t tpc = (cvec + kNT * ILP - 1) / (kNT * ILP);
       const uint64_t grid = tpc * (uint64_t)p;
       if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
-      rc_reduce_front_kernel<PMAX, TI, TO, OP, ILP><<<(unsigned)grid, kNT, 0, s>>>(a, tpc);
-      note_launches(1);
-      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+      if ((err = launch_kernel(rc_reduce_front_kernel<PMAX, TI, TO, OP, ILP>, dim3((unsigned)grid), dim3(kNT),
+                               0, s, a, tpc)) != cudaSuccess)
+        return err;
     }
     if (a.nvec * VEC < n) {
-      rc_reduce_tail_kernel<PMAX, TI, TO, OP><<<1, 32, 0, s>>>(a, a.nvec * VEC);
-      note_launches(1);
-      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+      if ((err = launch_kernel(rc_reduce_tail_kernel<PMAX, TI, TO, OP>, dim3(1), dim3(32), 0, s, a,
+                               a.nvec * VEC)) != cudaSuccess)
+        return err;
     }
   } else {
     auto kern = rc_reduce_scalar_kernel<PMAX, TI, TO, OP>;
@@ -244,9 +251,7 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
     a.nvec = n;
     uint64_t grid = std::min<uint64_t>((uint64_t)sms * std::max(occ, 1), (n + kNT - 1) / kNT);
     grid = std::max<uint64_t>(grid, 1);
-    kern<<<(unsigned)grid, kNT, 0, s>>>(a);
-    note_launches(1);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = launch_kernel(kern, dim3((unsigned)grid), dim3(kNT), 0, s, a)) != cudaSuccess) return err;
   }
   return cudaSuccess;
 }

@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "launch.cuh"
 
 namespace rc {
 namespace {
@@ -229,6 +230,8 @@ __global__ void __launch_bounds__(kRingNT, (PMAX <= 8 ? 4 : 2))
     }
   }
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
 
   const uint64_t G = gridDim.x;
   const uint64_t o0 = a.units * blockIdx.x / G;
@@ -343,9 +346,7 @@ cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   occ = std::max(1, std::min(occ, env_int("RC_CTAS_PER_SM", occ)));
   uint64_t grid = std::min<uint64_t>((uint64_t)sms * occ, (a.units + kRingNT - 1) / kRingNT);
   grid = std::max<uint64_t>(grid, 1);
-  kern<<<(unsigned)grid, kRingNT, 0, s>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kRingNT), 0, s, a);
 }
 
 template <class T, int OP>
