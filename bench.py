@@ -115,7 +115,7 @@ KERNEL_OF = {
     "all_gather": ("rc_fanout_bulk_kernel", "fanout.cu"),
     "reduce": ("rc_reduce_front_kernel", "reduce.cu"),
     "broadcast": ("rc_fanout_bulk_kernel", "fanout.cu"),
-    "ring_all_reduce": ("rc_ring_literal_kernel", "ring.cu"),
+    "ring_all_reduce": ("rc_ring_chain_kernel", "ring.cu"),
     "hier_all_reduce": ("rc_fold_tma_kernel", "fold.cu"),
 }
 

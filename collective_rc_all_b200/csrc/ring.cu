@@ -316,6 +316,156 @@ __global__ void __launch_bounds__(kRingNT, (PMAX <= 8 ? 4 : 2))
   }
 }
 
+// ---------------------------------------------------------------------------
+// Chain kernel (16-byte aligned buffers, chunks a whole number of vectors).
+//
+// The schedule above, regrouped: follow one chunk c through the ring.  Its
+// partial starts at rank c+1 (step 0 sends x_{c+1}[chunk c] to c+2), gains
+// x_d[chunk c] at each receiver d = c+k+2 (reduce-scatter step k), ends at
+// rank c after p-1 steps (d = c at step p-2, where it is scaled and cast
+// into y_c), and is then forwarded c -> c+1 -> ... -> c-1 by the all-gather
+// steps (step k: y_{c+k+1}[chunk c] = y_{c+k}[chunk c]).  Every message of
+// the schedule belongs to exactly one such chain, and different chunks'
+// chains never touch the same memory: the partial of chunk c at receiver d
+// lives in y_d[chunk c] (fp32 / int32), or for bf16 in the workspace slot
+// [k & 1][c] (two parities: the send buffer of step k-1 and the receive buffer
+// of step k are different memory).  So a thread can own CH chains of one
+// vector offset and run their 2(p-1) steps in program order, with no
+// synchronisation with the threads that own the other chains; the sends and
+// receives are real loads and stores of device memory as above.
+//
+// Each warp holds 32 consecutive offsets of the same chains, so every access
+// is a coalesced 512-byte row; the receivers' x values are loaded PF steps
+// ahead of the step that adds them.  The ranks of a step are warp-uniform:
+// their base pointers come from the kernel parameters.
+constexpr int kChainNT = 128;
+
+struct RingChainParams {
+  const char *x[kMaxRanks];
+  char *y[kMaxRanks];
+  char *ws;
+  uint64_t cv;  // vectors per chunk (C / VEC)
+  uint64_t nv;  // vectors in the whole per-rank vector (n / VEC)
+  float scale;
+  int p, ngroups;
+};
+
+template <class T, int OP, int CH, int PF>
+__global__ void __launch_bounds__(kChainNT) rc_ring_chain_kernel(const __grid_constant__ RingChainParams a) {
+  using Acc = typename T::Acc;
+  constexpr int VEC = kVec<T>;
+  constexpr int kIn = T::kBytes;
+  constexpr bool kWs = std::is_same<T, BF16>::value;
+  pdl_wait();
+  pdl_trigger();
+  const int p = a.p;
+  const uint64_t tile = blockIdx.x / (uint32_t)a.ngroups;
+  const int grp = (int)(blockIdx.x - tile * (uint32_t)a.ngroups);
+  const uint64_t o = tile * kChainNT + threadIdx.x;  // vector offset inside every chunk
+  const uint64_t cv = a.cv, C = cv * VEC;
+  const uint64_t oin = o * 16, o4 = o * (uint64_t)(VEC * 4);
+
+  int c[CH];          // this thread's chunks
+  bool on[CH];
+  uint64_t cin[CH];   // byte offset of chunk c in an input / output buffer
+  bool any = false;
+#pragma unroll
+  for (int i = 0; i < CH; ++i) {
+    c[i] = grp * CH + i;
+    const uint64_t b = (uint64_t)c[i] * cv;
+    const uint64_t len = (c[i] >= p || b >= a.nv) ? 0 : (a.nv - b < cv ? a.nv - b : cv);
+    on[i] = o < len;
+    any = any || on[i];
+    cin[i] = (uint64_t)c[i] * C * kIn;
+  }
+  if (!any) return;
+  auto wrap = [p](int v) { return v >= p ? v - p : v; };  // v < 2p
+  // partial of chunk c after step k, as received by d
+  auto part_at = [&](int i, int k, int d) -> char * {
+    if constexpr (kWs) return a.ws + ((uint64_t)((k & 1) * p + c[i])) * C * 4 + o4;
+    else return a.y[d] + cin[i] + o4;
+  };
+
+  // ---- reduce-scatter: p-1 steps; own[j][i] holds x of receiver c+k+2+j
+  uint4 own[PF][CH];
+  Acc acc[CH][VEC];
+#pragma unroll
+  for (int j = 0; j < PF; ++j) {
+#pragma unroll
+    for (int i = 0; i < CH; ++i)
+      if (on[i] && j < p - 1) own[j][i] = ld_cg_v4(a.x[wrap(wrap(c[i] + 2 + j))] + cin[i] + oin);
+  }
+#pragma unroll
+  for (int i = 0; i < CH; ++i)  // step 0's sends: x_{c+1}[chunk c]
+    if (on[i]) unpack<T>(ld_cg_v4(a.x[wrap(c[i] + 1)] + cin[i] + oin), acc[i]);
+  for (int k = 0; k + 1 < p; ++k) {
+    const bool last = (k + 2 == p);
+    if (k > 0) {
+#pragma unroll
+      for (int i = 0; i < CH; ++i)  // receive: the partial the previous step stored
+        if (on[i]) load_part<Acc, VEC, true>(part_at(i, k - 1, wrap(wrap(c[i] + k + 1))), acc[i]);
+    }
+    uint4 cur[CH];
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+      cur[i] = own[0][i];
+#pragma unroll
+      for (int j = 0; j + 1 < PF; ++j) own[j][i] = own[j + 1][i];
+      if (on[i] && k + PF < p - 1)  // x of the receiver PF steps ahead
+        own[PF - 1][i] = ld_cg_v4(a.x[wrap(wrap(c[i] + k + PF + 2))] + cin[i] + oin);
+    }
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+      if (!on[i]) continue;
+      Acc x[VEC];
+      unpack<T>(cur[i], x);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[i][e] = combine<OP>(acc[i][e], x[e]);
+      if (last) {  // the receiver is c itself: the finished chunk
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[i][e] = finish<OP>(acc[i][e], a.scale);
+        store_out<T, VEC>(a.y[c[i]] + cin[i] + oin, acc[i]);
+      } else {
+        store_part<Acc, VEC>(part_at(i, k, wrap(wrap(c[i] + k + 2))), acc[i]);
+      }
+    }
+  }
+
+  // ---- all-gather: p-1 steps, y_{c+k+1}[chunk c] = y_{c+k}[chunk c]
+  for (int k = 0; k + 1 < p; ++k) {
+    uint4 v[CH];
+#pragma unroll
+    for (int i = 0; i < CH; ++i)
+      if (on[i]) v[i] = ld_ca_v4(a.y[wrap(c[i] + k)] + cin[i] + oin);
+#pragma unroll
+    for (int i = 0; i < CH; ++i)
+      if (on[i]) st_v4(a.y[wrap(wrap(c[i] + k + 1))] + cin[i] + oin, v[i]);
+  }
+}
+
+template <class T, int OP, int CH, int PF>
+cudaError_t launch_ring_chain(const RingJob &job, uint64_t C, cudaStream_t s) {
+  RingChainParams a{};
+  const int p = job.p;
+  if (p < 2) return cudaErrorInvalidValue;  // no steps; the API never sends p = 1 here
+  constexpr int VEC = kVec<T>;
+  a.p = p;
+  a.cv = C / VEC;
+  a.nv = job.n / VEC;
+  a.scale = job.scale;
+  a.ws = static_cast<char *>(job.ws);
+  a.ngroups = (p + CH - 1) / CH;
+  for (int r = 0; r < p; ++r) {
+    a.x[r] = static_cast<const char *>(job.x[r]);
+    a.y[r] = static_cast<char *>(job.y[r]);
+  }
+  const uint64_t tiles = (a.cv + kChainNT - 1) / kChainNT;
+  const uint64_t grid = tiles * (uint64_t)a.ngroups;
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
+  return launch_kernel(rc_ring_chain_kernel<T, OP, CH, PF>, dim3((unsigned)grid), dim3(kChainNT), 0, s, a);
+}
+
 template <class T, int OP, int PMAX>
 cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   RingParams a{};
@@ -334,6 +484,16 @@ cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   }
   constexpr int VEC = kVec<T>;
   const bool vector = aligned && a.C % VEC == 0 && a.n % VEC == 0;
+  if (vector && env_int("RC_RING_KERNEL", 1) == 1) {
+    // default: 4 chains per thread, x one step ahead (72 registers, so that
+    // at p = 8 every offset's chains are resident at once); measured against
+    // 2 and 8 chains and a two-step prefetch.  RC_RING_KERNEL=0 selects the
+    // register kernel above on this path too.
+    const int ch = env_int("RC_RING_CH", 4), pf = env_int("RC_RING_PF", 1);
+    if (ch == 2) return pf == 1 ? launch_ring_chain<T, OP, 2, 1>(job, a.C, s) : launch_ring_chain<T, OP, 2, 2>(job, a.C, s);
+    if (ch == 8) return pf == 1 ? launch_ring_chain<T, OP, 8, 1>(job, a.C, s) : launch_ring_chain<T, OP, 8, 2>(job, a.C, s);
+    return pf == 1 ? launch_ring_chain<T, OP, 4, 1>(job, a.C, s) : launch_ring_chain<T, OP, 4, 2>(job, a.C, s);
+  }
   const int sms = device_sm_count();
   const bool l1 = env_int("RC_RING_L1", 1) != 0;
   auto kern = vector ? (l1 ? rc_ring_literal_kernel<T, OP, true, PMAX, true>
