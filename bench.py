@@ -69,10 +69,10 @@ WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 
 NCU_TRAFFIC = {
     # op: DRAM bytes per launch (read + write, one cold-cache ncu launch of the
     # step's workload), kernel source hash at capture time
-    "ring_all_reduce": {"bytes": 68177408 + 51077376, "src": "4d84d550ed796b2e"},
-    "all_reduce": {"bytes": 67133440 + 22459392, "src": "db7c2d49405fa2d0"},
-    "reduce_scatter": {"bytes": 67121408 + 987904, "src": "1a713eca9a1f13ac"},
-    "all_gather": {"bytes": 4205312 + 726528, "src": "216eaf2ee5963ca6"},
+    "ring_all_reduce": {"bytes": 67128320 + 33989888, "src": "79d77f64a1dae252"},
+    "all_reduce": {"bytes": 67130112 + 17357312, "src": "8395a3efc3921db4"},
+    "reduce_scatter": {"bytes": 67121408 + 1258752, "src": "2bfc7ab651598460"},
+    "all_gather": {"bytes": 4205312 + 196096, "src": "7c1e06d78d330fd4"},
 }
 
 
