@@ -52,9 +52,11 @@ def _bind(path: str) -> ctypes.CDLL:
     L.rco_bf16_to_f32.restype = ctypes.c_float
     L.rco_f32_to_bf16_n.argtypes = [ctypes.c_void_p, ctypes.c_void_p, sz]
     L.rco_f32_to_bf16_n.restype = None
+    fp = ctypes.POINTER(ctypes.c_float)
+    L.rco_adamw.argtypes = [fp, fp, fp, ctypes.c_void_p, ci, sz, cf, cf, cf, cf, cf, ctypes.c_int64]
     for f in ("rco_all_reduce", "rco_reduce_scatter", "rco_all_gather", "rco_reduce",
               "rco_broadcast", "rco_reduce_at", "rco_ring_all_reduce",
-              "rco_hier_all_reduce"):
+              "rco_hier_all_reduce", "rco_adamw"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -212,3 +214,67 @@ def f32_to_bf16(x: np.ndarray) -> np.ndarray:
 def bf16_to_f32(h: np.ndarray) -> np.ndarray:
     h = np.ascontiguousarray(h, dtype=np.uint16).ravel()
     return (h.astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- optimizer
+def adamw(theta, m, v, g, grad_dt="f32", lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8,
+          weight_decay=0.0, step=1):
+    """One AdamW step (rc_oracle.c rco_adamw); returns new (theta, m, v)."""
+    th = np.array(theta, dtype=np.float32, copy=True).ravel()
+    mm = np.array(m, dtype=np.float32, copy=True).ravel()
+    vv = np.array(v, dtype=np.float32, copy=True).ravel()
+    gg = np.ascontiguousarray(g, dtype=NP_DT[grad_dt]).ravel()
+    if not (th.size == mm.size == vv.size == gg.size):
+        raise ValueError("adamw: sizes differ")
+    fp = ctypes.POINTER(ctypes.c_float)
+    _check(lib().rco_adamw(th.ctypes.data_as(fp), mm.ctypes.data_as(fp), vv.ctypes.data_as(fp),
+                           gg.ctypes.data, DT[grad_dt], th.size, lr, beta1, beta2, eps,
+                           weight_decay, int(step)), "adamw")
+    return th, mm, vv
+
+
+def zero1_step(grads, master, exp_avg, exp_avg_sq, grad_dt="f32", param_dt="bf16",
+               scale=None, **hp):
+    """ZeRO-1 sharded optimizer step over p simulated ranks, by composition:
+    reduce_scatter of the gradients (fp32 out, x scale, default 1/p), AdamW on
+    each rank's own shard (fp32 master weights and moments of n/p elements),
+    then all_gather of the updated weights cast to param_dt.  Returns
+    (params per rank, master, exp_avg, exp_avg_sq) -- new arrays."""
+    p = len(grads)
+    if scale is None:
+        scale = 1.0 / p
+    g = reduce_scatter(grads, grad_dt, "f32", "sum", scale)
+    out_m, out_a, out_s = [], [], []
+    for r in range(p):
+        th, mm, vv = adamw(master[r], exp_avg[r], exp_avg_sq[r], g[r], "f32", **hp)
+        out_m.append(th)
+        out_a.append(mm)
+        out_s.append(vv)
+    shards = [th if param_dt == "f32" else f32_to_bf16(th) for th in out_m]
+    return all_gather(shards, param_dt), out_m, out_a, out_s
+
+
+def sharded_owner_step(grads, master, exp_avg, exp_avg_sq, grad_dt="f32", param_dt="bf16",
+                       scale=None, **hp):
+    """The ShardedOptimizer form: tensor t (lists of per-rank arrays) is owned
+    by rank t % p; every gradient is all-reduced (x scale, default 1/p), the
+    owner runs AdamW on its fp32 master copy and moments, and the result is
+    broadcast from the owner.  grads[t][r]: rank r's gradient of tensor t;
+    master / exp_avg / exp_avg_sq[t]: the owner's state of tensor t.
+    Returns (params[t][r], master, exp_avg, exp_avg_sq) -- new arrays."""
+    T = len(grads)
+    p = len(grads[0])
+    if scale is None:
+        scale = 1.0 / p
+    params, out_m, out_a, out_s = [], [], [], []
+    for t in range(T):
+        owner = t % p
+        g = all_reduce(grads[t], grad_dt, "sum", scale)
+        g32 = g[owner] if grad_dt == "f32" else bf16_to_f32(g[owner])
+        th, mm, vv = adamw(master[t], exp_avg[t], exp_avg_sq[t], g32, "f32", **hp)
+        out_m.append(th)
+        out_a.append(mm)
+        out_s.append(vv)
+        w = th if param_dt == "f32" else f32_to_bf16(th)
+        params.append(broadcast(w, p, owner, param_dt))
+    return params, out_m, out_a, out_s

@@ -27,6 +27,12 @@
  *            own matching chunk; after N-1 steps card 0 holds chunk 0 ...),
  *            phase 2 all-gather (each card forwards its finished chunk to the
  *            next card, which overwrites), 2(N-1) steps in total.
+ *  [P2-ZERO] "分布式训练/推理", sections "DDP 模型训练示例" (ShardedOptimizer:
+ *            average the gradients, run AdamW on the parameters this rank owns,
+ *            broadcast every parameter from its owner) and "显存账：不同数据并行的
+ *            局限性" (ZeRO-1 shards the optimizer state: the Adam moments and the
+ *            fp32 master weights).  The pages name torch.optim.AdamW without
+ *            printing it; the update below is AdamW's published definition.
  *  [P1-HIER] "大模型并行的最小闭环：集合通信、TP、FSDP/ZeRO-3 到权重分片", log excerpt
  *            "分层 AllReduce + SHARP": 2 nodes x 4 GPUs, B per GPU; step 1 intra-node
  *            AllReduce, step 2 one representative (GPU0) per node, step 3 uplink B
@@ -50,11 +56,16 @@
  *     step is a ring over the group (so its order is R1 with q = G); the
  *     leader (local rank 0) sums the group results in ring order over the
  *     groups (q = p/G); scale and cast happen once, after the leader sum.
+ *  R6 AdamW (rco_adamw): binary32, each operation rounded once, in the order
+ *     written there; the scalars 1 - lr*wd, 1 - beta1, 1 - beta2, 1 - beta1^t
+ *     and 1 - beta2^t are evaluated in binary64 (the C library's pow) and
+ *     rounded to binary32 once.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math (oracle/build.py).
  * x86-64 float arithmetic is SSE binary32, so every `float` operation below is
  * one correctly rounded IEEE operation.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -583,5 +594,44 @@ int rco_hier_all_reduce(const void *const *send, void *const *recv, int p, int G
     for (int g = 0; g < ng; ++g)
         free(S[g]);
     free(S);
+    return RCO_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* AdamW, one step on n elements [P2-ZERO], in place.                        */
+/* Definition (decoupled weight decay, bias-corrected moments), step t >= 1:  */
+/*   theta <- theta * (1 - lr*wd)                                            */
+/*   m     <- beta1*m + (1 - beta1)*g                                        */
+/*   v     <- beta2*v + (1 - beta2)*(g*g)                                    */
+/*   mhat  <- m / (1 - beta1^t)          vhat <- v / (1 - beta2^t)            */
+/*   theta <- theta - lr * (mhat / (sqrt(vhat) + eps))                       */
+/* Reading R6: every line is evaluated left to right in binary32, one        */
+/* rounding per operation; the five scalars in parentheses that do not       */
+/* involve m, v, g or theta are binary64 expressions rounded once.            */
+/* g is fp32 (grad_dt RCO_F32) or bf16 bits (RCO_BF16), widened exactly.      */
+int rco_adamw(float *theta, float *m, float *v, const void *g, int grad_dt, size_t n,
+              float lr, float beta1, float beta2, float eps, float wd, int64_t t)
+{
+    if (t < 1 || (grad_dt != RCO_F32 && grad_dt != RCO_BF16))
+        return RCO_EINVAL;
+    const float decay = (float)(1.0 - (double)lr * (double)wd);
+    const float omb1 = (float)(1.0 - (double)beta1);
+    const float omb2 = (float)(1.0 - (double)beta2);
+    const float bc1 = (float)(1.0 - pow((double)beta1, (double)t));
+    const float bc2 = (float)(1.0 - pow((double)beta2, (double)t));
+    for (size_t i = 0; i < n; ++i) {
+        float gi = grad_dt == RCO_F32 ? ((const float *)g)[i]
+                                      : rco_bf16_to_f32(((const uint16_t *)g)[i]);
+        float th = theta[i] * decay;
+        float mi = beta1 * m[i] + omb1 * gi;
+        float vi = beta2 * v[i] + omb2 * (gi * gi);
+        float mhat = mi / bc1;
+        float vhat = vi / bc2;
+        float den = sqrtf(vhat) + eps;
+        th = th - lr * (mhat / den);
+        theta[i] = th;
+        m[i] = mi;
+        v[i] = vi;
+    }
     return RCO_OK;
 }

@@ -33,6 +33,14 @@ MUTANTS = {
     "ring_receiver_operands_swapped": [("combine(msg[r][i - b], w[d][i], is_int, op)", "combine(w[d][i], msg[r][i - b], is_int, op)")],
     "ring_allgather_wrong_chunk": [("size_t c = (size_t)(((r - k) % p + p) % p);", "size_t c = (size_t)(((r - k - 1) % p + p) % p);")],
     "hier_group_drops_a_rank": [("ring_core(send + (size_t)g * (size_t)G, G,", "ring_core(send + (size_t)g * (size_t)G, G > 1 ? G - 1 : G,")],
+    "adamw_no_first_bias_correction": [("float mhat = mi / bc1;", "float mhat = mi;")],
+    "adamw_eps_inside_sqrt": [("float den = sqrtf(vhat) + eps;", "float den = sqrtf(vhat + eps);")],
+    "adamw_decay_after_update": [("float th = theta[i] * decay;", "float th = theta[i];"),
+                                 ("th = th - lr * (mhat / den);", "th = (th - lr * (mhat / den)) * decay;")],
+    "adamw_second_moment_of_g_not_g2": [("float vi = beta2 * v[i] + omb2 * (gi * gi);",
+                                         "float vi = beta2 * v[i] + omb2 * gi;")],
+    "adamw_update_sign_flipped": [("th = th - lr * (mhat / den);", "th = th + lr * (mhat / den);")],
+    "adamw_betas_swapped": [("float mi = beta1 * m[i] + omb1 * gi;", "float mi = beta2 * m[i] + omb2 * gi;")],
     "int_sum_saturates": [("acc.i = (int32_t)((uint32_t)acc.i + (uint32_t)v.i);",
                            "{ long long t = (long long)acc.i + v.i; acc.i = t > 2147483647LL ? 2147483647 : (t < -2147483648LL ? (int32_t)-2147483648LL : (int32_t)t); }")],
 }
@@ -49,9 +57,10 @@ def test_pins_catch_planted_mistake(name):
         so = os.path.join(d, "libmutant.so")
         open(c, "w").write(src)
         subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-                        "-o", so, c], check=True)
+                        "-o", so, c, "-lm"], check=True)
         env = dict(os.environ, RC_ORACLE_LIB=so)
         r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                            os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                            os.path.join(ROOT, "tests", "test_oracle_optim.py")],
                            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
