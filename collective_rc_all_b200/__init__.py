@@ -65,6 +65,17 @@ _decl("rc_ring_all_reduce", [_vpp, _vpp, _i, _sz, _i, _i, _f, _i, _vp])
 _decl("rc_hier_all_reduce", [_vpp, _vpp, _i, _i, _sz, _i, _i, _f, _i, _vp])
 _decl("rc_ring_all_reduce_noalloc", [_vpp, _vpp, _i, _sz, _i, _i, _f, _vp])
 _decl("rc_copy", [_vp, _vp, _sz, _vp])
+
+
+class rc_adamw_hparams(ctypes.Structure):
+    """Mirror of the C struct rc_adamw_hparams."""
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
+
+
+_hpp = ctypes.POINTER(rc_adamw_hparams)
+_decl("rc_adamw_step", [_vp, _vp, _vp, _vp, _i, _sz, _hpp, _vp])
+_decl("rc_zero1_step", [_vpp, _vpp, _vpp, _vpp, _vpp, _i, _sz, _i, _i, _f, _hpp, _vp])
 _decl("rc_reserve_workspace", [_sz, _vp])
 _decl("rc_check_buffer", [_vp, _sz])
 _decl("rc_probe_bounded_wait", [ctypes.c_uint64, _vp])
@@ -214,6 +225,30 @@ def rc_hier_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], group_size: int
     _check(lib.rc_hier_all_reduce(_ptrs(send), _ptrs(recv), p, group_size, _numel(send[0], n),
                                   _dt(dtype, send[0]), _op(op), scale, int(v), _stream(stream)),
            "rc_hier_all_reduce")
+
+
+def _hparams(lr, beta1, beta2, eps, weight_decay, step):
+    return rc_adamw_hparams(lr, beta1, beta2, eps, weight_decay, int(step))
+
+
+def rc_adamw_step(param: Buf, exp_avg: Buf, exp_avg_sq: Buf, grad: Buf, n=None, grad_dtype=None,
+                  lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1, stream=None):
+    hp = _hparams(lr, beta1, beta2, eps, weight_decay, step)
+    _check(lib.rc_adamw_step(_addr(param), _addr(exp_avg), _addr(exp_avg_sq), _addr(grad),
+                             _dt(grad_dtype, grad), _numel(param, n), ctypes.byref(hp),
+                             _stream(stream)), "rc_adamw_step")
+
+
+def rc_zero1_step(grads: Sequence[Buf], params: Sequence[Buf], master: Sequence[Buf],
+                  exp_avg: Sequence[Buf], exp_avg_sq: Sequence[Buf], n=None, grad_dtype=None,
+                  param_dtype=None, scale=None, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8,
+                  weight_decay=0.0, step=1, stream=None):
+    p = len(grads)
+    hp = _hparams(lr, beta1, beta2, eps, weight_decay, step)
+    _check(lib.rc_zero1_step(_ptrs(grads), _ptrs(params), _ptrs(master), _ptrs(exp_avg),
+                             _ptrs(exp_avg_sq), p, _numel(grads[0], n), _dt(grad_dtype, grads[0]),
+                             _dt(param_dtype, params[0]), 1.0 / p if scale is None else scale,
+                             ctypes.byref(hp), _stream(stream)), "rc_zero1_step")
 
 
 def rc_copy(src: Buf, dst: Buf, nbytes=None, stream=None):

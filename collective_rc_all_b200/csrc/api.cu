@@ -164,6 +164,9 @@ rc_status check_aliasing(const std::vector<Buf> &bs) {
 
 rc_status check_ranges(const std::vector<Buf> &bs) {
   for (const Buf &b : bs) {
+    if (b.esz > 1 && b.lo % (uintptr_t)b.esz != 0)
+      return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p is not aligned to its %d-byte elements", b.what, b.idx,
+                  (void *)b.lo, b.esz);
     rc_status st = check_device_range((const void *)b.lo, b.hi - b.lo, b.what, b.idx);
     if (st != RC_OK) return st;
   }
@@ -524,6 +527,85 @@ rc_status rc_hier_all_reduce(const void *const *send, void *const *recv, int p, 
   st = launched(launch_hier_staged(j, (cudaStream_t)stream), "hier staged launch");
   ws_release(dev, (cudaStream_t)stream);
   return st;
+}
+
+namespace {
+rc_status check_hparams(const rc_adamw_hparams *hp, AdamwHyper *out) {
+  if (!hp) return fail(RC_ERR_INVALID_ARG, "hparams is NULL");
+  if (hp->step < 1) return fail(RC_ERR_INVALID_ARG, "step=%lld must be >= 1", (long long)hp->step);
+  out->lr = hp->lr;
+  out->beta1 = hp->beta1;
+  out->beta2 = hp->beta2;
+  out->eps = hp->eps;
+  out->weight_decay = hp->weight_decay;
+  out->step = hp->step;
+  return RC_OK;
+}
+bool float_dt_ok(int d) { return d == RC_FP32 || d == RC_BF16; }
+}  // namespace
+
+rc_status rc_adamw_step(float *param, float *exp_avg, float *exp_avg_sq, const void *grad,
+                        rc_dtype grad_dt, size_t n, const rc_adamw_hparams *hp, rc_stream_t stream) {
+  rc_status st;
+  AdamwHyper h{};
+  if ((st = check_hparams(hp, &h)) != RC_OK) return st;
+  if (!float_dt_ok(grad_dt)) return fail(RC_ERR_INVALID_ARG, "grad dtype must be fp32 or bf16");
+  if (n > kMaxElems) return fail(RC_ERR_INVALID_ARG, "n=%zu too large", n);
+  if (n == 0) return RC_OK;
+  std::vector<Buf> bs;
+  bs.push_back(make_buf(grad, n, dt_size(grad_dt), 0, 0, false, "grad", 0));
+  bs.push_back(make_buf(param, n, 4, 0, 1, true, "param", 0));
+  bs.push_back(make_buf(exp_avg, n, 4, 0, 2, true, "exp_avg", 0));
+  bs.push_back(make_buf(exp_avg_sq, n, 4, 0, 3, true, "exp_avg_sq", 0));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  return launched(launch_adamw(param, exp_avg, exp_avg_sq, grad, grad_dt, n, h, (cudaStream_t)stream),
+                  "adamw launch");
+}
+
+rc_status rc_zero1_step(const void *const *grads, void *const *params, float *const *master,
+                        float *const *exp_avg, float *const *exp_avg_sq, int p, size_t n,
+                        rc_dtype grad_dt, rc_dtype param_dt, float scale,
+                        const rc_adamw_hparams *hp, rc_stream_t stream) {
+  rc_status st;
+  AdamwHyper h{};
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_hparams(hp, &h)) != RC_OK) return st;
+  if (!float_dt_ok(grad_dt) || !float_dt_ok(param_dt))
+    return fail(RC_ERR_INVALID_ARG, "grad and param dtypes must be fp32 or bf16");
+  if (n % (size_t)p != 0) return fail(RC_ERR_INVALID_ARG, "n=%zu is not a multiple of p=%d", n, p);
+  if (n == 0) return RC_OK;
+  if (!grads || !params || !master || !exp_avg || !exp_avg_sq)
+    return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const uint64_t m = n / p;
+  std::vector<Buf> bs;
+  // ranks 0..p-1 for the gradients and parameters; the three state arrays of
+  // rank r get their own "rank" ids so that no in-place overlap with a
+  // gradient or parameter buffer is accepted
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(grads[r], n, dt_size(grad_dt), 0, r, false, "grads", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(params[r], n, dt_size(param_dt), 0, r, true, "params", r));
+  for (int r = 0; r < p; ++r) {
+    bs.push_back(make_buf(master[r], m, 4, 0, kMaxP + 3 * r, true, "master", r));
+    bs.push_back(make_buf(exp_avg[r], m, 4, 0, kMaxP + 3 * r + 1, true, "exp_avg", r));
+    bs.push_back(make_buf(exp_avg_sq[r], m, 4, 0, kMaxP + 3 * r + 2, true, "exp_avg_sq", r));
+  }
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  Zero1Job j{};
+  j.p = p;
+  j.n = n;
+  for (int r = 0; r < p; ++r) {
+    j.grad[r] = grads[r];
+    j.param[r] = params[r];
+    j.master[r] = master[r];
+    j.exp_avg[r] = exp_avg[r];
+    j.exp_avg_sq[r] = exp_avg_sq[r];
+  }
+  j.grad_dt = grad_dt;
+  j.param_dt = param_dt;
+  j.scale = scale;
+  j.hp = h;
+  return launched(launch_zero1(j, (cudaStream_t)stream), "zero1 launch");
 }
 
 rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream) {

@@ -71,6 +71,27 @@ struct HierJob {
   float scale;
 };
 
+// AdamW hyperparameters of one step (optim.cu).
+struct AdamwHyper {
+  float lr, beta1, beta2, eps, weight_decay;
+  int64_t step;  // t >= 1
+};
+
+// ZeRO-1 step over p ranks (optim.cu): gradients in, full parameters out on
+// every rank, fp32 master weights and moments sharded (rank r: n/p elements).
+struct Zero1Job {
+  const void *grad[kMaxP];
+  void *param[kMaxP];
+  float *master[kMaxP];
+  float *exp_avg[kMaxP];
+  float *exp_avg_sq[kMaxP];
+  int p;
+  uint64_t n;
+  int grad_dt, param_dt;
+  float scale;
+  AdamwHyper hp;
+};
+
 cudaError_t launch_reduce(const ReduceJob &job, cudaStream_t s);
 bool fold_tma_eligible(const FoldJob &job);
 cudaError_t launch_fold_tma(const FoldJob &job, cudaStream_t s);
@@ -82,6 +103,9 @@ cudaError_t noalloc_scratch_ptr(void **out);
 cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s);
 cudaError_t launch_hier_staged(const HierJob &job, cudaStream_t s);
 cudaError_t launch_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);
+cudaError_t launch_zero1(const Zero1Job &job, cudaStream_t s);
+cudaError_t launch_adamw(float *param, float *exp_avg, float *exp_avg_sq, const void *grad, int grad_dt,
+                         uint64_t n, const AdamwHyper &hp, cudaStream_t s);
 
 cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s);
 

@@ -26,6 +26,12 @@
  *         of N-1 steps (send one chunk to the next card, which accumulates);
  *         all-gather phase of N-1 steps (forward the finished chunk, receiver
  *         overwrites); 2(N-1) steps; card 0 ends the first phase holding chunk 0.
+ *  [ZERO] "分布式训练/推理", section "显存账：不同数据并行的局限性" -- ZeRO-1
+ *         shards the optimizer state (Adam moments, fp32 master weights) while
+ *         every rank keeps full parameters; section "DDP 模型训练示例" -- the
+ *         ShardedOptimizer averages the gradients, runs AdamW on the parameters
+ *         its rank owns and hands every rank the owner's parameters.  The page
+ *         names torch.optim.AdamW without printing it (see rc_adamw_step).
  *  [HIER] "大模型并行的最小闭环：集合通信、TP、FSDP/ZeRO-3 到权重分片", log excerpt
  *         "分层 AllReduce + SHARP", steps 1-6 -- intra-node AllReduce, one
  *         representative per node, the node results added together, intra-node
@@ -194,6 +200,58 @@ rc_status rc_ring_all_reduce_noalloc(const void *const *send, void *const *recv,
 rc_status rc_hier_all_reduce(const void *const *send, void *const *recv, int p, int group_size,
                              size_t n, rc_dtype dt, rc_op op, float scale,
                              rc_hier_variant variant, rc_stream_t stream);
+
+/* AdamW hyperparameters of one optimizer step [ZERO]. */
+typedef struct rc_adamw_hparams {
+  float lr;
+  float beta1;
+  float beta2;
+  float eps;
+  float weight_decay;
+  int64_t step; /* t >= 1: the index of this step (bias corrections use it) */
+} rc_adamw_hparams;
+
+/*
+ * One AdamW step on n elements, in place: [ZERO] names torch.optim.AdamW; the
+ * update is AdamW's published definition (decoupled weight decay,
+ * bias-corrected moments), evaluated in binary32 with one rounding per
+ * operation in exactly this order:
+ *   theta <- theta * (1 - lr*wd)
+ *   m     <- beta1*m + (1 - beta1)*g
+ *   v     <- beta2*v + (1 - beta2)*(g*g)
+ *   mhat  <- m / (1 - beta1^t);   vhat <- v / (1 - beta2^t)
+ *   theta <- theta - lr * (mhat / (sqrt(vhat) + eps))
+ * The scalars 1 - lr*wd, 1 - beta1, 1 - beta2, 1 - beta1^t, 1 - beta2^t are
+ * binary64 expressions (C library pow) rounded to binary32 once.
+ *  param, exp_avg, exp_avg_sq: n fp32 each, read and written.
+ *  grad: n elements of grad_dt (RC_FP32 or RC_BF16, widened exactly), read.
+ *  The four buffers must not overlap.  hp->step < 1, a NULL hp or another
+ *  grad_dt return RC_ERR_INVALID_ARG.
+ */
+rc_status rc_adamw_step(float *param, float *exp_avg, float *exp_avg_sq, const void *grad,
+                        rc_dtype grad_dt, size_t n, const rc_adamw_hparams *hp, rc_stream_t stream);
+
+/*
+ * ZeRO-1 sharded optimizer step [ZERO], [FSDP], [AVG], fused with its
+ * collectives in one pass over p simulated ranks (n % p == 0, m = n/p):
+ *   g[i]         = scale * (fold of grads[0..p-1][i] in the ring order of
+ *                  chunk c = i / m), fp32 accumulate  (the reduce-scatter:
+ *                  rank c owns shard c; scale is typically 1/p)
+ *   shard c      : rc_adamw_step's update of master[c][j], exp_avg[c][j],
+ *                  exp_avg_sq[c][j] with g[c*m + j], j < m
+ *   params[q][i] = cast_param(master[c][i - c*m]) for every rank q (the
+ *                  all-gather; bf16 is round-to-nearest-even)
+ * Bit-identical to rc_reduce_scatter (fp32 out) + rc_adamw_step per shard +
+ * rc_all_gather.
+ *  grads[r]: n elements of grad_dt (RC_FP32 / RC_BF16), read.
+ *  params[q]: n elements of param_dt (RC_FP32 / RC_BF16), written.
+ *  master[r], exp_avg[r], exp_avg_sq[r]: m fp32 each (rank r's shard), read
+ *  and written.  Output and state buffers must not overlap one another.
+ */
+rc_status rc_zero1_step(const void *const *grads, void *const *params, float *const *master,
+                        float *const *exp_avg, float *const *exp_avg_sq, int p, size_t n,
+                        rc_dtype grad_dt, rc_dtype param_dt, float scale,
+                        const rc_adamw_hparams *hp, rc_stream_t stream);
 
 /*
  * Plain device copy dst[0, bytes) = src[0, bytes) with this library's

@@ -16,7 +16,11 @@ reproduction recipe state them):
   * uniform[lo, hi), normal N(0, sigma) (sigma is a standard deviation),
     integers uniform[lo, hi);
   * the transformer-layer parameter count 4*4096*4096 + 3*4096*11008 of a
-    Llama-2-7B decoder layer (Q, K, V, O projections and gate, up, down).
+    Llama-2-7B decoder layer (Q, K, V, O projections and gate, up, down);
+  * optimizer state for the sharded AdamW step: fp32 master weights
+    uniform[-1, 1), first moments N(0, 1e-3), second moments the squares of
+    an N(0, 1e-3) draw, each split into p shards; the step's hyperparameters
+    (ZERO1_ADAMW) are a synthetic recipe, since the pages give none.
 """
 from __future__ import annotations
 
@@ -30,6 +34,9 @@ import torch
 LLAMA2_7B_LAYER_ELEMS = 4 * 4096 * 4096 + 3 * 4096 * 11008  # 202,375,168
 
 NP = {"f32": np.float32, "bf16": np.uint16, "i32": np.int32}
+
+# AdamW hyperparameters of the sharded-optimizer workload (synthetic recipe).
+ZERO1_ADAMW = dict(lr=3e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, step=10)
 
 
 def _gen(seed: int) -> torch.Generator:
@@ -113,6 +120,7 @@ def config(name: str):
         "cfg3_hier": dict(p=8, n=4194304, dt="bf16", gen="normal", seed=2, sigma=1.0, group=4),
         "cfg4_params": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS // 8, dt="bf16", gen="uniform", seed=3),
         "cfg4_grads": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS, dt="f32", gen="normal", seed=4, sigma=1e-3),
+        "zero1_state": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS, gen="adam_state", seed=5),
     }
     return cfgs[name]
 
@@ -125,4 +133,18 @@ def draw(cfg: dict) -> List[np.ndarray]:
         return uniform(cfg["p"], cfg["n"], cfg["seed"], cfg["dt"])
     if g == "normal":
         return normal(cfg["p"], cfg["n"], cfg["seed"], cfg.get("sigma", 1.0), cfg["dt"])
+    if g == "adam_state":
+        return adam_state(cfg["p"], cfg["n"], cfg["seed"])
     raise ValueError(g)
+
+
+def adam_state(p: int, n: int, seed: int):
+    """(master, exp_avg, exp_avg_sq): three lists of p fp32 shards of n // p
+    elements -- master uniform[-1, 1), exp_avg N(0, 1e-3), exp_avg_sq the
+    squares of an N(0, 1e-3) draw -- from one generator, in that order."""
+    g = _gen(seed)
+    m = n // p
+    master = [(torch.rand(m, generator=g, dtype=torch.float32) * 2 - 1).numpy() for _ in range(p)]
+    ea = [(torch.randn(m, generator=g, dtype=torch.float32) * 1e-3).numpy() for _ in range(p)]
+    es = [(torch.randn(m, generator=g, dtype=torch.float32) * 1e-3).square().numpy() for _ in range(p)]
+    return master, ea, es

@@ -92,3 +92,24 @@ def test_host_memory_is_not_a_device_pointer(rc):
     before = rc.rc_launch_count()
     assert rc.lib.rc_all_reduce(ptr, ptr, 2, 64, 0, 0, 1.0, None) == 1
     assert rc.rc_launch_count() == before
+
+
+def test_optimizer_arguments_rejected_on_host(rc):
+    L = rc.lib
+    a = _null(8)
+    hp = rc.rc_adamw_hparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+    bad_step = rc.rc_adamw_hparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 0)
+    before = rc.rc_launch_count()
+    assert L.rc_zero1_step(a, a, a, a, a, 8, 64, 0, 1, 0.125, None, None) == 1           # NULL hparams
+    assert L.rc_zero1_step(a, a, a, a, a, 8, 64, 0, 1, 0.125, ctypes.byref(bad_step), None) == 1
+    assert L.rc_zero1_step(a, a, a, a, a, 8, 60, 0, 1, 0.125, ctypes.byref(hp), None) == 1  # 8 does not divide 60
+    assert L.rc_zero1_step(a, a, a, a, a, 8, 64, 2, 1, 0.125, ctypes.byref(hp), None) == 1  # int32 grads
+    assert L.rc_zero1_step(a, a, a, a, a, 8, 64, 0, 2, 0.125, ctypes.byref(hp), None) == 1  # int32 params
+    assert L.rc_zero1_step(a, a, a, a, a, 17, 64, 0, 1, 0.125, ctypes.byref(hp), None) == 1  # p > 16
+    assert L.rc_zero1_step(a, a, a, a, a, 8, 64, 0, 1, 0.125, ctypes.byref(hp), None) == 1  # NULL buffers
+    assert L.rc_adamw_step(None, None, None, None, 0, 16, None, None) == 1
+    assert L.rc_adamw_step(None, None, None, None, 2, 16, ctypes.byref(hp), None) == 1      # int32 grad
+    assert L.rc_adamw_step(None, None, None, None, 0, 16, ctypes.byref(hp), None) == 1      # NULL buffers
+    assert L.rc_zero1_step(a, a, a, a, a, 8, 0, 0, 1, 0.125, ctypes.byref(hp), None) == 0   # empty
+    assert L.rc_adamw_step(None, None, None, None, 0, 0, ctypes.byref(hp), None) == 0
+    assert rc.rc_launch_count() == before
