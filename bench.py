@@ -684,6 +684,126 @@ def run_sweep(args):
     return 0
 
 
+def zero1_bytes(p: int, n: int, s_grad: int, s_param: int) -> int:
+    """Minimum bytes of one ZeRO-1 step over p ranks of n elements: every
+    gradient read once, the fp32 master weights and both moments read and
+    written once, every rank's parameters written once."""
+    return p * n * s_grad + 2 * 3 * 4 * n + p * n * s_param
+
+
+def run_zero1(args):
+    """The sharded-optimizer workload (one JSON line): the ZeRO-1 AdamW step on
+    a Llama-2-7B decoder layer (202,375,168 parameters) over 8 simulated
+    ranks, fp32 gradients ~N(0, 1e-3), fp32 master weights and moments
+    sharded 1/8 per rank.  Variants, each timed with CUDA events over K
+    back-to-back steps after W warm-ups (every buffer is far larger than L2):
+      fused_bf16     rc_zero1_step, bf16 parameters (the workload)
+      fused_f32      rc_zero1_step, fp32 parameters
+      unfused_f32    rc_reduce_scatter (fp32, x 1/8) + rc_adamw_step per
+                     shard + rc_all_gather of the fp32 master shards
+      owner_f32      the ShardedOptimizer form: per weight tensor, in-place
+                     rc_all_reduce (x 1/8), rc_adamw_step by the owner
+                     (tensor t % 8), rc_broadcast from the owner
+    Effective GB/s always uses the fused step's minimum bytes (zero1_bytes)."""
+    import torch
+    import collective_rc_all_b200 as rc
+    import rc_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    p, N = 8, args.zero1_elems
+    if N % (8 * 4096) != 0:
+        raise SystemExit("--zero1-elems must be a multiple of 8 * 4096")
+    m = N // p
+    hp = dict(rc_inputs.ZERO1_ADAMW)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    grads = [torch.randn(N, generator=gen, device=dev) * 1e-3 for _ in range(p)]
+    gen.manual_seed(5)
+    master = [torch.rand(m, generator=gen, device=dev) * 2 - 1 for _ in range(p)]
+    ea = [torch.randn(m, generator=gen, device=dev) * 1e-3 for _ in range(p)]
+    es = [(torch.randn(m, generator=gen, device=dev) * 1e-3).square() for _ in range(p)]
+    p_bf16 = [torch.empty(N, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+    p_f32 = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(p)]
+    gs = [torch.empty(m, dtype=torch.float32, device=dev) for _ in range(p)]
+    # owner form: full-size fp32 state per tensor on its owner (views of flat arrays)
+    shapes = [4096 * 4096] * 4 + [4096 * 11008] * 3
+    if N != sum(shapes):  # a scaled-down case (profiling): the same seven tensors, scaled
+        shapes = [s * N // sum(shapes) for s in shapes]
+        shapes[-1] += N - sum(shapes)
+    o_master = torch.rand(N, generator=gen, device=dev) * 2 - 1
+    o_ea = torch.zeros(N, device=dev)
+    o_es = torch.zeros(N, device=dev)
+    offs = np.concatenate([[0], np.cumsum(shapes)]).astype(np.int64)
+
+    def owner_step():
+        for t, s in enumerate(shapes):
+            a, b = int(offs[t]), int(offs[t + 1])
+            gt = [g[a:b] for g in grads]
+            owner = t % p
+            rc.rc_all_reduce(gt, gt, scale=1.0 / p)
+            rc.rc_adamw_step(o_master[a:b], o_ea[a:b], o_es[a:b], gt[owner], **hp)
+            outs = [q[a:b] for q in p_f32]
+            outs[owner] = o_master[a:b]
+            rc.rc_broadcast(o_master[a:b], outs, root=owner)
+
+    def unfused_step():
+        rc.rc_reduce_scatter(grads, gs, out_dtype="f32", scale=1.0 / p)
+        for r in range(p):
+            rc.rc_adamw_step(master[r], ea[r], es[r], gs[r], **hp)
+        rc.rc_all_gather(master, p_f32)
+
+    variants = {
+        "fused_bf16": (lambda: rc.rc_zero1_step(grads, p_bf16, master, ea, es, param_dtype="bf16", **hp), 2),
+        "fused_f32": (lambda: rc.rc_zero1_step(grads, p_f32, master, ea, es, param_dtype="f32", **hp), 4),
+        "unfused_f32": (unfused_step, 4),
+        "owner_f32": (owner_step, 4),
+    }
+    K, W = args.steps, args.warmup
+    peak, peak_kind = measured_peaks()
+    res = {}
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    for name, (fn, sp) in variants.items():
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        l0 = rc.rc_launch_count()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        t = a.elapsed_time(b) * 1e-3 / K
+        byt = zero1_bytes(p, N, 4, sp)
+        res[name] = {"ms": round(t * 1e3, 4), "min_bytes": byt, "gbs": round(byt / t / 1e9, 1),
+                     "frac_of_measured_hbm": round(byt / t / 1e9 / peak, 4),
+                     "launches_per_step": (rc.rc_launch_count() - l0) // K}
+    clk = clocks.stop()
+    rc.rc_stream_status()
+    f = res["fused_bf16"]
+    line = {
+        "metric": "effective GB/s of the fused ZeRO-1 AdamW step (reduce-scatter, AdamW, all-gather in one pass)",
+        "value": f["gbs"], "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": f["ms"], "higher_is_better": True, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"ZeRO-1 AdamW step, {N:,} parameters (202,375,168 = one Llama-2-7B decoder layer), "
+                               "p=8 simulated ranks, fp32 gradients ~N(0,1e-3), fp32 master weights "
+                               "uniform[-1,1) and moments sharded 1/8, bf16 parameters on every rank",
+                   "adamw": hp, "l2": "inputs larger than L2 (GBs per step)"},
+        "roofline": {"bound": "hbm", "kernel": "rc_zero1_front_kernel", "achieved": f["gbs"], "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": f["frac_of_measured_hbm"],
+                     "algorithmic_bytes": f["min_bytes"]},
+        "variants": res,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -704,12 +824,18 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--sweep-max-bytes", type=int, default=1 << 30)
     ap.add_argument("--sweep-out", default="")
+    # the sharded-optimizer workload (ZeRO-1 AdamW step): one JSON line
+    ap.add_argument("--zero1", action="store_true")
+    ap.add_argument("--zero1-elems", type=int, default=202375168,
+                    help="parameters of the ZeRO-1 workload (default: one Llama-2-7B decoder layer)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.zero1:
+        return run_zero1(args)
     return run_ours(args)
 
 

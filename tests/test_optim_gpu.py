@@ -86,6 +86,14 @@ def test_zero1_step_matches_oracle(rc, p, grad_dt, param_dt):
     _zero1_case(rc, p, p * (3 * 2048 + 40), grad_dt, param_dt, seed=40 + p)
 
 
+@pytest.mark.parametrize("p,param_dt", [(8, "bf16"), (3, "bf16"), (8, "f32")])
+def test_zero1_odd_vector_count_per_shard(rc, p, param_dt):
+    """m = 4 * 1001: an odd number of 16-byte vectors per shard, so every other
+    shard starts off a 16-byte boundary of the bf16 parameters and the last
+    thread of a shard holds a single vector."""
+    _zero1_case(rc, p, p * 4 * 1001, "f32", param_dt, seed=60 + p)
+
+
 @pytest.mark.parametrize("p,n,offset", [(8, 8 * 1001, 0), (4, 4 * 6, 0), (8, 8 * 512, 4), (3, 3 * 333, 0)])
 def test_zero1_element_path(rc, p, n, offset):
     """Shard lengths that are not whole vectors, and buffers off a 16-byte
@@ -168,3 +176,33 @@ def test_zero1_llama_layer_sampled(rc):
     for q in (0, 3, p - 1):
         got = pd[q].index_select(0, ti).view(torch.int16).cpu().numpy().view(np.uint16)
         assert_bits(got, want_p, f"llama zero1 params rank {q} (sampled)")
+
+
+def test_sharded_owner_broadcast_variant(rc):
+    """The ShardedOptimizer form through library calls: every gradient tensor
+    all-reduced with scale 1/p, AdamW by the owner (tensor t % p) on its fp32
+    master copy, the result broadcast from the owner; against the oracle."""
+    p, sizes = 4, [5, 4096, 1, 333, 8, 1 << 14]
+    r = np.random.default_rng(31)
+    grads = [[(r.standard_normal(s) * 1e-3).astype(np.float32) for _ in range(p)] for s in sizes]
+    master = [r.uniform(-1, 1, s).astype(np.float32) for s in sizes]
+    ea = [(r.standard_normal(s) * 1e-3).astype(np.float32) for s in sizes]
+    es = [np.square(r.standard_normal(s) * 1e-3).astype(np.float32) for s in sizes]
+    want, w_m, w_a, w_s = oracle.sharded_owner_step(grads, master, ea, es, param_dt="f32", **HP)
+    for t, s in enumerate(sizes):
+        owner = t % p
+        gd, _ = to_dev(grads[t], "f32")
+        rc.rc_all_reduce(gd, gd, scale=1.0 / p)  # in place, like dist.all_reduce(AVG)
+        (th,), _ = to_dev([master[t]], "f32")
+        (mm,), _ = to_dev([ea[t]], "f32")
+        (vv,), _ = to_dev([es[t]], "f32")
+        rc.rc_adamw_step(th, mm, vv, gd[owner], **HP)
+        out, _ = empty_dev(s, "f32", p)
+        out[owner] = th  # the owner's own copy is the updated master (broadcast in place)
+        rc.rc_broadcast(th, out, root=owner)
+        _sync(rc)
+        assert_bits(to_host(th, "f32"), w_m[t], f"owner master t={t}")
+        assert_bits(to_host(mm, "f32"), w_a[t], f"owner exp_avg t={t}")
+        assert_bits(to_host(vv, "f32"), w_s[t], f"owner exp_avg_sq t={t}")
+        for q in range(p):
+            assert_bits(to_host(out[q], "f32"), want[t][q], f"owner broadcast t={t} rank {q}")
