@@ -54,9 +54,10 @@ def _bind(path: str) -> ctypes.CDLL:
     L.rco_f32_to_bf16_n.restype = None
     fp = ctypes.POINTER(ctypes.c_float)
     L.rco_adamw.argtypes = [fp, fp, fp, ctypes.c_void_p, ci, sz, cf, cf, cf, cf, cf, ctypes.c_int64]
+    L.rco_all_to_all_v.argtypes = [vpp, vpp, ci, u64p, ci, u64p]
     for f in ("rco_all_reduce", "rco_reduce_scatter", "rco_all_gather", "rco_reduce",
               "rco_broadcast", "rco_reduce_at", "rco_ring_all_reduce",
-              "rco_hier_all_reduce", "rco_adamw"):
+              "rco_hier_all_reduce", "rco_adamw", "rco_all_to_all_v"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -278,3 +279,36 @@ def sharded_owner_step(grads, master, exp_avg, exp_avg_sq, grad_dt="f32", param_
         w = th if param_dt == "f32" else f32_to_bf16(th)
         params.append(broadcast(w, p, owner, param_dt))
     return params, out_m, out_a, out_s
+
+
+# ---------------------------------------------------------------- all-to-all
+def all_to_all_v(sends, counts, traffic=None):
+    """sends[r]: rank r's outgoing blocks in destination order; counts[r][q]:
+    elements r sends to q (any numpy dtype, copied bit for bit).  Returns the
+    p receive buffers (incoming blocks in source order).  traffic, if a list
+    of 2, gets [bytes staying on their rank, bytes crossing ranks] added."""
+    p = len(sends)
+    cnt = np.ascontiguousarray(counts, dtype=np.uint64).reshape(p, p)
+    dt = sends[0].dtype
+    xs = [np.ascontiguousarray(x) for x in sends]
+    for r in range(p):
+        if xs[r].dtype != dt or xs[r].size < int(cnt[r].sum()):
+            raise ValueError("all_to_all_v: send buffer too short or of another dtype")
+    outs = [np.empty(int(cnt[:, q].sum()), dt) for q in range(p)]
+    tr = np.zeros(2, np.uint64)
+    u64p = ctypes.POINTER(ctypes.c_uint64)
+    _check(lib().rco_all_to_all_v(_ptrs(xs), _ptrs(outs), p, cnt.ctypes.data_as(u64p), dt.itemsize,
+                                  tr.ctypes.data_as(u64p)), "all_to_all_v")
+    if traffic is not None:
+        traffic[0] += int(tr[0])
+        traffic[1] += int(tr[1])
+    return outs
+
+
+def all_to_all(sends, traffic=None):
+    """Equal splits: n = p*m elements per rank, block q of rank r -> slot r of rank q."""
+    p = len(sends)
+    n = sends[0].size
+    if n % p:
+        raise ValueError("all_to_all: n must be a multiple of p")
+    return all_to_all_v(sends, np.full((p, p), n // p, np.uint64), traffic)

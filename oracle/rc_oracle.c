@@ -33,6 +33,13 @@
  *            局限性" (ZeRO-1 shards the optimizer state: the Adam moments and the
  *            fp32 master weights).  The pages name torch.optim.AdamW without
  *            printing it; the update below is AdamW's published definition.
+ *  [P2-A2A]  "分布式训练/推理", primitive table: all-to-all -- every rank sends a
+ *            different slice to every rank (MoE token routing); section "从路由
+ *            结果到专家输出" (dispatch = the exchange towards the experts, combine
+ *            = the way back; split counts tell a receiver how much arrives) and
+ *            section "为什么 top-k 和 EP degree 会直接放大通信" (payload t*k*h*b
+ *            per phase, of which t*k*h*b*(p-1)/p leaves the rank when routing is
+ *            balanced).
  *  [P1-HIER] "大模型并行的最小闭环：集合通信、TP、FSDP/ZeRO-3 到权重分片", log excerpt
  *            "分层 AllReduce + SHARP": 2 nodes x 4 GPUs, B per GPU; step 1 intra-node
  *            AllReduce, step 2 one representative (GPU0) per node, step 3 uplink B
@@ -632,6 +639,37 @@ int rco_adamw(float *theta, float *m, float *v, const void *g, int grad_dt, size
         theta[i] = th;
         m[i] = mi;
         v[i] = vi;
+    }
+    return RCO_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* all-to-all with split counts [P2-A2A].                                     */
+/* counts[r*p + q] = elements rank r sends to rank q.  Rank r's send buffer   */
+/* holds its p outgoing blocks in destination order q = 0..p-1; rank q's      */
+/* receive buffer holds its p incoming blocks in source order r = 0..p-1:     */
+/*   send offset of block (r,q) = sum_{q' < q} counts[r*p + q']                */
+/*   recv offset of block (r,q) = sum_{r' < r} counts[r'*p + q]                */
+/* Each block is copied bit for bit.  traffic (optional, 2 counters, bytes):  */
+/* [0] blocks that stay on their rank (r == q), [1] blocks that cross ranks.  */
+int rco_all_to_all_v(const void *const *send, void *const *recv, int p, const uint64_t *counts,
+                     int esz, uint64_t *traffic)
+{
+    if (p < 1 || p > 64 || (esz != 1 && esz != 2 && esz != 4 && esz != 8) || !counts)
+        return RCO_EINVAL;
+    for (int r = 0; r < p; ++r) {
+        for (int q = 0; q < p; ++q) {
+            uint64_t soff = 0, roff = 0;
+            for (int k = 0; k < q; ++k)
+                soff += counts[(size_t)r * p + k];
+            for (int k = 0; k < r; ++k)
+                roff += counts[(size_t)k * p + q];
+            uint64_t c = counts[(size_t)r * p + q];
+            memcpy((char *)recv[q] + roff * (uint64_t)esz, (const char *)send[r] + soff * (uint64_t)esz,
+                   c * (uint64_t)esz);
+            if (traffic)
+                traffic[r == q ? 0 : 1] += c * (uint64_t)esz;
+        }
     }
     return RCO_OK;
 }

@@ -41,6 +41,12 @@ MUTANTS = {
                                          "float vi = beta2 * v[i] + omb2 * gi;")],
     "adamw_update_sign_flipped": [("th = th - lr * (mhat / den);", "th = th + lr * (mhat / den);")],
     "adamw_betas_swapped": [("float mi = beta1 * m[i] + omb1 * gi;", "float mi = beta2 * m[i] + omb2 * gi;")],
+    "a2a_recv_offset_by_destination": [("for (int k = 0; k < r; ++k)\n                roff += counts[(size_t)k * p + q];",
+                                        "for (int k = 0; k < q; ++k)\n                roff += counts[(size_t)r * p + k];")],
+    "a2a_send_offset_off_by_one": [("for (int k = 0; k < q; ++k)\n                soff += counts[(size_t)r * p + k];",
+                                    "for (int k = 0; k <= q && k < p - 1; ++k)\n                soff += counts[(size_t)r * p + k];")],
+    "a2a_transposed_count": [("uint64_t c = counts[(size_t)r * p + q];", "uint64_t c = counts[(size_t)q * p + r];")],
+    "a2a_traffic_swapped": [("traffic[r == q ? 0 : 1] += c * (uint64_t)esz;", "traffic[r == q ? 1 : 0] += c * (uint64_t)esz;")],
     "int_sum_saturates": [("acc.i = (int32_t)((uint32_t)acc.i + (uint32_t)v.i);",
                            "{ long long t = (long long)acc.i + v.i; acc.i = t > 2147483647LL ? 2147483647 : (t < -2147483648LL ? (int32_t)-2147483648LL : (int32_t)t); }")],
 }
@@ -61,6 +67,7 @@ def test_pins_catch_planted_mistake(name):
         env = dict(os.environ, RC_ORACLE_LIB=so)
         r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                             os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                            os.path.join(ROOT, "tests", "test_oracle_optim.py")],
+                            os.path.join(ROOT, "tests", "test_oracle_optim.py"),
+                            os.path.join(ROOT, "tests", "test_oracle_a2a.py")],
                            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
