@@ -3,6 +3,7 @@ plausible slip, builds the copy, and runs the pin tests against it.  Every
 slip must make the pins fail -- otherwise the pins could not tell a wrong
 oracle from a right one.  CPU only; the real oracle is never modified.
 """
+import concurrent.futures
 import os
 import subprocess
 import sys
@@ -52,11 +53,12 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name):
+def _run_mutant(name):
+    """Build one mutant and run the pins against it; returns (returncode, tail of output)."""
     src = open(SRC).read()
     for old, new in MUTANTS[name]:
-        assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+        if src.count(old) < 1:
+            return None, f"mutation anchor not found: {old!r}"
         src = src.replace(old, new)
     with tempfile.TemporaryDirectory() as d:
         c = os.path.join(d, "mutant.c")
@@ -65,9 +67,29 @@ def test_pins_catch_planted_mistake(name):
         subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
                         "-o", so, c, "-lm"], check=True)
         env = dict(os.environ, RC_ORACLE_LIB=so)
-        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                            os.path.join(ROOT, "tests", "test_oracle_optim.py"),
-                            os.path.join(ROOT, "tests", "test_oracle_a2a.py")],
+        # the pin file that covers the mutated function runs first, so that a
+        # caught mutant stops at its first failure
+        pins = ["test_oracle_pins.py", "test_oracle_optim.py", "test_oracle_a2a.py"]
+        first = ("test_oracle_optim.py" if name.startswith("adamw") else
+                 "test_oracle_a2a.py" if name.startswith("a2a") else "test_oracle_pins.py")
+        pins.remove(first)
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"] +
+                           [os.path.join(ROOT, "tests", f) for f in [first] + pins],
                            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results():
+    """All mutants, built and checked in parallel (independent processes)."""
+    workers = max(1, min(8, (os.cpu_count() or 2)))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        futs = {n: ex.submit(_run_mutant, n) for n in MUTANTS}
+        return {n: f.result() for n, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, mutant_results):
+    rc, out = mutant_results[name]
+    assert rc is not None, out
+    assert rc != 0, f"pins did not catch mutant {name}:\n{out}"
