@@ -804,6 +804,110 @@ def run_zero1(args):
     return 0
 
 
+def moe_counts(p: int, t: int, k: int, experts: int, seed: int, zipf: float) -> np.ndarray:
+    """Token-expert assignments per (source rank, destination rank) of one MoE
+    layer: every rank routes t tokens to k distinct experts each, expert e
+    lives on rank e // (experts // p), expert popularity ~ 1 / rank^zipf
+    (zipf = 0: uniform).  Returns a p x p array of assignment counts."""
+    rng = np.random.default_rng(seed)
+    w = 1.0 / np.arange(1, experts + 1) ** zipf
+    w = w[rng.permutation(experts)]
+    w /= w.sum()
+    per_rank = experts // p
+    c = np.zeros((p, p), np.int64)
+    for r in range(p):
+        for _ in range(t):
+            e = rng.choice(experts, size=k, replace=False, p=w)
+            for x in e:
+                c[r, x // per_rank] += 1
+    return c
+
+
+def run_a2a(args):
+    """The MoE dispatch/combine workload (one JSON line): 8 simulated ranks
+    (EP group), t = 4096 tokens per rank, top-2 routing, hidden 4096, bf16
+    activations -- t*k*h*b = 64 MiB per rank and phase.  Variants: balanced
+    routing (rc_all_to_all, equal splits) and skewed routing over 64 experts
+    with popularity ~ 1/rank^1.2 (rc_all_to_all_v); each times the dispatch
+    and the combine (the same exchange with the transposed counts) with CUDA
+    events over K back-to-back rounds after W warm-ups.  Effective GB/s =
+    (bytes read + written) / time; the cross-rank payload is reported too."""
+    import torch
+    import collective_rc_all_b200 as rc
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    p, t, k, h, E = 8, 4096, 2, 4096, 64
+    b = 2
+    peak, peak_kind = measured_peaks()
+    K, W = args.steps, args.warmup
+    res = {}
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    for name, zipf in (("balanced", None), ("skewed", 1.2)):
+        if zipf is None:
+            tok = np.full((p, p), t * k // p, np.int64)
+        else:
+            tok = moe_counts(p, t, k, E, seed=7, zipf=zipf)
+        counts = tok * h
+        send = [torch.empty(int(counts[r].sum()), dtype=torch.bfloat16, device=dev).normal_() for r in range(p)]
+        mid = [torch.empty(int(counts[:, q].sum()), dtype=torch.bfloat16, device=dev) for q in range(p)]
+        back = [torch.empty(int(counts[r].sum()), dtype=torch.bfloat16, device=dev) for r in range(p)]
+        if zipf is None:
+            dispatch = lambda: rc.rc_all_to_all(send, mid)
+            combine = lambda: rc.rc_all_to_all(mid, back)
+        else:
+            dispatch = lambda: rc.rc_all_to_all_v(send, mid, counts)
+            combine = lambda: rc.rc_all_to_all_v(mid, back, counts.T)
+        for _ in range(W):
+            dispatch()
+            combine()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
+        for i in range(K):
+            ev[2 * i].record(stream)
+            dispatch()
+            ev[2 * i + 1].record(stream)
+            combine()
+        ev[-1].record(stream)
+        ev[-1].synchronize()
+        td = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)) * 1e-3 / K
+        tc = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(K)) * 1e-3 / K
+        payload = int(counts.sum()) * b                  # all blocks, one phase
+        cross = int(counts.sum() - np.trace(counts)) * b  # blocks that change rank
+        res[name] = {
+            "dispatch_us": round(td * 1e6, 2), "combine_us": round(tc * 1e6, 2),
+            "payload_bytes_per_phase": payload, "cross_rank_bytes_per_phase": cross,
+            "max_rank_recv_bytes": int(counts.sum(axis=0).max()) * b,
+            "dispatch_gbs": round(2 * payload / td / 1e9, 1), "combine_gbs": round(2 * payload / tc / 1e9, 1),
+            "dispatch_frac_of_measured_hbm": round(2 * payload / td / 1e9 / peak, 4),
+            "tokens_per_pair": tok.tolist() if zipf is not None else int(tok[0, 0]),
+        }
+        del send, mid, back
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    rc.rc_stream_status()
+    bal = res["balanced"]
+    line = {
+        "metric": "effective GB/s of the MoE all-to-all dispatch (bytes read + written / time)",
+        "value": bal["dispatch_gbs"], "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": round((bal["dispatch_us"] + bal["combine_us"]) / 1e3, 4), "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "MoE dispatch + combine: p=8 simulated ranks, t=4096 tokens per rank, top-2, "
+                               "hidden 4096, bf16 (t*k*h*b = 64 MiB per rank and phase); skewed: 64 experts, "
+                               "popularity ~ 1/rank^1.2, seed 7", "l2": "inputs larger than L2 (512 MiB per phase)"},
+        "roofline": {"bound": "hbm", "kernel": "rc_a2a_kernel", "achieved": bal["dispatch_gbs"], "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": bal["dispatch_frac_of_measured_hbm"],
+                     "algorithmic_bytes": 2 * bal["payload_bytes_per_phase"]},
+        "variants": res,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -826,6 +930,8 @@ def main(argv=None):
     ap.add_argument("--sweep-out", default="")
     # the sharded-optimizer workload (ZeRO-1 AdamW step): one JSON line
     ap.add_argument("--zero1", action="store_true")
+    # the MoE dispatch / combine workload (all-to-all): one JSON line
+    ap.add_argument("--a2a", action="store_true")
     ap.add_argument("--zero1-elems", type=int, default=202375168,
                     help="parameters of the ZeRO-1 workload (default: one Llama-2-7B decoder layer)")
     args = ap.parse_args(argv)
@@ -836,6 +942,8 @@ def main(argv=None):
         return run_sweep(args)
     if args.zero1:
         return run_zero1(args)
+    if args.a2a:
+        return run_a2a(args)
     return run_ours(args)
 
 

@@ -76,6 +76,8 @@ class rc_adamw_hparams(ctypes.Structure):
 _hpp = ctypes.POINTER(rc_adamw_hparams)
 _decl("rc_adamw_step", [_vp, _vp, _vp, _vp, _i, _sz, _hpp, _vp])
 _decl("rc_zero1_step", [_vpp, _vpp, _vpp, _vpp, _vpp, _i, _sz, _i, _i, _f, _hpp, _vp])
+_decl("rc_all_to_all", [_vpp, _vpp, _i, _sz, _i, _vp])
+_decl("rc_all_to_all_v", [_vpp, _vpp, _i, ctypes.POINTER(ctypes.c_size_t), _i, _vp])
 _decl("rc_reserve_workspace", [_sz, _vp])
 _decl("rc_check_buffer", [_vp, _sz])
 _decl("rc_probe_bounded_wait", [ctypes.c_uint64, _vp])
@@ -249,6 +251,23 @@ def rc_zero1_step(grads: Sequence[Buf], params: Sequence[Buf], master: Sequence[
                              _ptrs(exp_avg_sq), p, _numel(grads[0], n), _dt(grad_dtype, grads[0]),
                              _dt(param_dtype, params[0]), 1.0 / p if scale is None else scale,
                              ctypes.byref(hp), _stream(stream)), "rc_zero1_step")
+
+
+def rc_all_to_all(send: Sequence[Buf], recv: Sequence[Buf], n=None, dtype=None, stream=None):
+    p = len(send)
+    _check(lib.rc_all_to_all(_ptrs(send), _ptrs(recv), p, _numel(send[0], n), _dt(dtype, send[0]),
+                             _stream(stream)), "rc_all_to_all")
+
+
+def rc_all_to_all_v(send: Sequence[Buf], recv: Sequence[Buf], counts, dtype=None, stream=None):
+    """counts: p x p element counts (nested sequence or array), counts[r][q] = r -> q."""
+    p = len(send)
+    flat = [int(c) for row in counts for c in row]
+    if len(flat) != p * p:
+        raise ValueError("counts must be p x p")
+    arr = (ctypes.c_size_t * (p * p))(*flat)
+    _check(lib.rc_all_to_all_v(_ptrs(send), _ptrs(recv), p, arr, _dt(dtype, send[0]), _stream(stream)),
+           "rc_all_to_all_v")
 
 
 def rc_copy(src: Buf, dst: Buf, nbytes=None, stream=None):

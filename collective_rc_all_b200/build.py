@@ -21,6 +21,7 @@ CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "librankcoll.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+EXPORTS = os.path.join(HERE, "exports.map")  # only the C ABI (rc_*) is exported
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # -fmad=false: no contraction of a*b+c (the fold is adds and one multiply, and
@@ -71,9 +72,10 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
     objs = [os.path.join(OBJ, os.path.basename(s)[:-3] + ".o") for s in srcs]
-    if force or jobs or _stale(LIB, objs):
+    if force or jobs or _stale(LIB, objs + [EXPORTS]):
         tmp = LIB + ".tmp"
-        subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], check=True)
+        subprocess.run([nvcc(), *ARCH, "-shared", "-Xlinker", f"--version-script={EXPORTS}", "-o", tmp, *objs],
+                       check=True)
         os.replace(tmp, LIB)
     return LIB
 

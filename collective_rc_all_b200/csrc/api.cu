@@ -608,6 +608,58 @@ rc_status rc_zero1_step(const void *const *grads, void *const *params, float *co
   return launched(launch_zero1(j, (cudaStream_t)stream), "zero1 launch");
 }
 
+rc_status rc_all_to_all_v(const void *const *send, void *const *recv, int p, const size_t *counts,
+                          rc_dtype dt, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, 0)) != RC_OK) return st;
+  if (!dt_ok(dt)) return fail(RC_ERR_INVALID_ARG, "unknown dtype");
+  if (!counts) return fail(RC_ERR_INVALID_ARG, "counts is NULL");
+  uint64_t total = 0;
+  std::vector<uint64_t> sent(p, 0), got(p, 0);
+  for (int r = 0; r < p; ++r)
+    for (int q = 0; q < p; ++q) {
+      const uint64_t c = counts[(size_t)r * p + q];
+      if (c > kMaxElems) return fail(RC_ERR_INVALID_ARG, "counts[%d][%d]=%llu too large", r, q,
+                                     (unsigned long long)c);
+      sent[r] += c;
+      got[q] += c;
+      total += c;
+    }
+  for (int r = 0; r < p; ++r)
+    if (sent[r] > kMaxElems || got[r] > kMaxElems)
+      return fail(RC_ERR_INVALID_ARG, "rank %d sends or receives too many elements", r);
+  if (total == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  // sends and receives get distinct "ranks": no overlap between them is
+  // accepted (a rank's incoming blocks would overwrite outgoing ones)
+  for (int r = 0; r < p; ++r)
+    if (sent[r]) bs.push_back(make_buf(send[r], sent[r], s, 0, r, false, "send", r));
+  for (int q = 0; q < p; ++q)
+    if (got[q]) bs.push_back(make_buf(recv[q], got[q], s, 0, kMaxP + q, true, "recv", q));
+  if ((st = check_ranges(bs)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  A2aJob j{};
+  j.p = p;
+  j.esz = s;
+  for (int r = 0; r < p; ++r) {
+    j.send[r] = send[r];
+    j.recv[r] = recv[r];
+  }
+  for (int i = 0; i < p * p; ++i) j.counts[i] = counts[i];
+  return launched(launch_all_to_all(j, (cudaStream_t)stream), "all_to_all launch");
+}
+
+rc_status rc_all_to_all(const void *const *send, void *const *recv, int p, size_t n, rc_dtype dt,
+                        rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if (n % (size_t)p != 0) return fail(RC_ERR_INVALID_ARG, "n=%zu is not a multiple of p=%d", n, p);
+  std::vector<size_t> counts((size_t)p * p, n / p);
+  return rc_all_to_all_v(send, recv, p, counts.data(), dt, stream);
+}
+
 rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream) {
   if (bytes == 0) return RC_OK;
   rc_status st;

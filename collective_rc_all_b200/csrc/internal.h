@@ -92,6 +92,16 @@ struct Zero1Job {
   AdamwHyper hp;
 };
 
+// All-to-all with split counts (alltoall.cu): counts[r*p + q] elements of
+// esz bytes go from rank r to rank q.
+struct A2aJob {
+  const void *send[kMaxP];
+  void *recv[kMaxP];
+  uint64_t counts[kMaxP * kMaxP];
+  int p;
+  int esz;
+};
+
 cudaError_t launch_reduce(const ReduceJob &job, cudaStream_t s);
 bool fold_tma_eligible(const FoldJob &job);
 cudaError_t launch_fold_tma(const FoldJob &job, cudaStream_t s);
@@ -104,6 +114,7 @@ cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s);
 cudaError_t launch_hier_staged(const HierJob &job, cudaStream_t s);
 cudaError_t launch_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);
 cudaError_t launch_zero1(const Zero1Job &job, cudaStream_t s);
+cudaError_t launch_all_to_all(const A2aJob &job, cudaStream_t s);
 cudaError_t launch_adamw(float *param, float *exp_avg, float *exp_avg_sq, const void *grad, int grad_dt,
                          uint64_t n, const AdamwHyper &hp, cudaStream_t s);
 

@@ -32,6 +32,11 @@
  *         ShardedOptimizer averages the gradients, runs AdamW on the parameters
  *         its rank owns and hands every rank the owner's parameters.  The page
  *         names torch.optim.AdamW without printing it (see rc_adamw_step).
+ *  [A2A]  "分布式训练/推理", primitive table -- all-to-all: every rank sends a
+ *         different slice to every rank (MoE token routing); section "从路由结果
+ *         到专家输出" -- dispatch towards the experts and combine back, split
+ *         counts tell the receiver how much arrives; section "为什么 top-k 和 EP
+ *         degree 会直接放大通信" -- payload t*k*h*b per rank and phase.
  *  [HIER] "大模型并行的最小闭环：集合通信、TP、FSDP/ZeRO-3 到权重分片", log excerpt
  *         "分层 AllReduce + SHARP", steps 1-6 -- intra-node AllReduce, one
  *         representative per node, the node results added together, intra-node
@@ -200,6 +205,27 @@ rc_status rc_ring_all_reduce_noalloc(const void *const *send, void *const *recv,
 rc_status rc_hier_all_reduce(const void *const *send, void *const *recv, int p, int group_size,
                              size_t n, rc_dtype dt, rc_op op, float scale,
                              rc_hier_variant variant, rc_stream_t stream);
+
+/*
+ * All-to-all with split counts [A2A] (MoE dispatch; the combine is the same
+ * call with the transposed counts).  counts is a host array of p*p element
+ * counts, row-major: counts[r*p + q] elements go from rank r to rank q.
+ *  send[r]: rank r's outgoing blocks in destination order q = 0..p-1
+ *           (sum_q counts[r*p+q] elements), read.
+ *  recv[q]: rank q's incoming blocks in source order r = 0..p-1
+ *           (sum_r counts[r*p+q] elements), written.
+ * Block (r, q) is copied bit for bit from send[r] + sum_{q'<q} counts[r*p+q']
+ * to recv[q] + sum_{r'<r} counts[r'*p+q].  Any dtype (elements are copied).
+ * No send buffer may overlap a receive buffer; receive buffers must not
+ * overlap one another.  All counts zero: RC_OK, nothing launched.
+ */
+rc_status rc_all_to_all_v(const void *const *send, void *const *recv, int p, const size_t *counts,
+                          rc_dtype dt, rc_stream_t stream);
+
+/* Equal splits: n elements per rank (n % p == 0), counts[r*p+q] = n/p, i.e.
+ * recv[q][r*(n/p) + j] = send[r][q*(n/p) + j]. */
+rc_status rc_all_to_all(const void *const *send, void *const *recv, int p, size_t n, rc_dtype dt,
+                        rc_stream_t stream);
 
 /* AdamW hyperparameters of one optimizer step [ZERO]. */
 typedef struct rc_adamw_hparams {
