@@ -908,6 +908,121 @@ def run_a2a(args):
     return 0
 
 
+def run_ddp(args):
+    """The DDP gradient-synchronisation workload (one JSON line): 8 simulated
+    ranks, two Llama-2-7B decoder layers (9 tensors each: W_q, W_k, W_v, W_o,
+    W_gate, W_up, W_down and two norm weights), bf16 gradients in one flat
+    buffer per rank in backward order.  A synthetic backward computes each
+    rank's weight gradients as X^T dY (cuBLAS bf16 GEMMs, T tokens per rank)
+    straight into the flat buffers, last tensor first, on the compute stream;
+    the gradient bucketer averages them (x 1/8) on a high-priority
+    communication stream.  Strategies of the pages' comparison:
+      none           backward only (the reference time)
+      naive          per-tensor all-reduce, all issued after backward
+      flat_after     one all-reduce of everything after backward
+      per_tensor     per-tensor all-reduce as soon as each gradient is ready
+      bucket_25mb    25 MiB buckets as soon as each bucket is complete
+    Reported per strategy (CUDA events, mean of K steps after W warm-ups):
+    step time, backward time, and the exposed tail = end of the last
+    all-reduce - end of backward."""
+    import torch
+    import collective_rc_all_b200 as rc
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    main_s = torch.cuda.current_stream()
+    comm = torch.cuda.Stream(priority=-1)
+    p, L, T, h, f = 8, 2, args.ddp_tokens, 4096, 11008
+    layer = [("norm1", (h,)), ("q", (h, h)), ("k", (h, h)), ("v", (h, h)), ("o", (h, h)),
+             ("norm2", (h,)), ("gate", (h, f)), ("up", (h, f)), ("down", (f, h))]
+    fwd = [(f"l{l}.{nm}", shp) for l in range(L) for nm, shp in layer]
+    bwd = fwd[::-1]                                       # gradients become ready in this order
+    numel = [int(np.prod(s_)) for _, s_ in bwd]
+    off = np.concatenate([[0], np.cumsum(numel)]).astype(np.int64)
+    N = int(off[-1])
+    grads = [torch.zeros(N, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    X = [torch.randn(T, f, generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(p)]
+    dY = [torch.randn(T, f, generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(p)]
+
+    def grad_of(t, r):
+        nm, shp = bwd[t]
+        view = grads[r][int(off[t]):int(off[t + 1])]
+        if len(shp) == 1:   # norm weight: sum over tokens of x * dy
+            torch.sum(X[r][:, :h] * dY[r][:, :h], dim=0, out=view)
+        else:               # weight (in, out): X[:, :in]^T @ dY[:, :out]
+            torch.matmul(X[r][:, :shp[0]].t(), dY[r][:, :shp[1]], out=view.view(shp))
+
+    strategies = {"none": None, "naive": (0, False), "flat_after": (2 ** 63, False),
+                  "per_tensor": (0, True), "bucket_25mb": (25 << 20, True)}
+    K, W = args.steps, args.warmup
+    res = {}
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    for name, cfg in strategies.items():
+        b = None if cfg is None else rc.Bucketer(grads, numel, cfg[0], comm_stream=comm)
+        nb = len(b.buckets()) if b else 0
+
+        def step():
+            l0 = rc.rc_launch_count()
+            for t in range(len(bwd)):
+                for r in range(p):
+                    grad_of(t, r)
+                if b is not None and cfg[1]:
+                    b.ready(t, main_s)
+            e_bwd = torch.cuda.Event(enable_timing=True)
+            e_bwd.record(main_s)
+            if b is not None and not cfg[1]:
+                for t in range(len(bwd)):
+                    b.ready(t, main_s)
+            if b is not None:
+                b.flush(main_s)
+            return e_bwd, rc.rc_launch_count() - l0
+
+        for _ in range(W):
+            step()
+        torch.cuda.synchronize()
+        tot, bw, launches = [], [], 0
+        for _ in range(K):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(main_s)
+            e_bwd, nl = step()
+            e1.record(main_s)
+            e1.synchronize()
+            tot.append(e0.elapsed_time(e1))
+            bw.append(e0.elapsed_time(e_bwd))
+            launches = nl
+        rc.rc_stream_status()
+        res[name] = {"step_ms": round(float(np.mean(tot)), 4), "backward_ms": round(float(np.mean(bw)), 4),
+                     "exposed_tail_ms": round(float(np.mean(tot) - np.mean(bw)), 4),
+                     "buckets": nb, "all_reduce_kernels_per_step": int(launches)}
+        if b is not None:
+            b.close()
+    clk = clocks.stop()
+    base = res["none"]["step_ms"]
+    for r_ in res.values():
+        r_["slowdown_vs_backward_only"] = round(r_["step_ms"] / base, 4)
+    ar_bytes = 2 * p * N * 2   # every gradient read and written once by the reduction
+    best = min((k for k in res if k != "none"), key=lambda k: res[k]["step_ms"])
+    line = {
+        "metric": "exposed gradient-communication tail after backward, DDP bucketing strategies",
+        "value": res[best]["exposed_tail_ms"], "unit": "ms", "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": res[best]["step_ms"], "higher_is_better": False, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"DDP gradient sync: p=8 simulated ranks, 2 Llama-2-7B decoder layers "
+                               f"({N:,} parameters, 18 tensors), bf16 gradients from X^T dY GEMMs with "
+                               f"T={T} tokens per rank, average (x 1/8) by bucketed in-place all-reduce on a "
+                               f"high-priority stream", "best": best,
+                   "all_reduce_bytes_per_step": ar_bytes},
+        "strategies": res,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -932,6 +1047,9 @@ def main(argv=None):
     ap.add_argument("--zero1", action="store_true")
     # the MoE dispatch / combine workload (all-to-all): one JSON line
     ap.add_argument("--a2a", action="store_true")
+    # the DDP gradient-bucketing workload: one JSON line
+    ap.add_argument("--ddp", action="store_true")
+    ap.add_argument("--ddp-tokens", type=int, default=1024, help="tokens per rank of the synthetic backward")
     ap.add_argument("--zero1-elems", type=int, default=202375168,
                     help="parameters of the ZeRO-1 workload (default: one Llama-2-7B decoder layer)")
     args = ap.parse_args(argv)
@@ -944,6 +1062,8 @@ def main(argv=None):
         return run_zero1(args)
     if args.a2a:
         return run_a2a(args)
+    if args.ddp:
+        return run_ddp(args)
     return run_ours(args)
 
 

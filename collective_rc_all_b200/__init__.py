@@ -77,6 +77,15 @@ _hpp = ctypes.POINTER(rc_adamw_hparams)
 _decl("rc_adamw_step", [_vp, _vp, _vp, _vp, _i, _sz, _hpp, _vp])
 _decl("rc_zero1_step", [_vpp, _vpp, _vpp, _vpp, _vpp, _i, _sz, _i, _i, _f, _hpp, _vp])
 _decl("rc_all_to_all", [_vpp, _vpp, _i, _sz, _i, _vp])
+_szp = ctypes.POINTER(ctypes.c_size_t)
+_ip = ctypes.POINTER(ctypes.c_int)
+_decl("rc_plan_buckets", [_i, _szp, _sz, _sz, _ip, _ip])
+_decl("rc_bucketer_create", [ctypes.POINTER(_vp), _vpp, _i, _i, _szp, _sz, _i, _f, _vp])
+_decl("rc_bucketer_num_buckets", [_vp, _ip])
+_decl("rc_bucketer_bucket", [_vp, _i, _ip, _ip, _szp, _szp])
+_decl("rc_bucketer_ready", [_vp, _i, _vp])
+_decl("rc_bucketer_flush", [_vp, _vp])
+_decl("rc_bucketer_destroy", [_vp])
 _decl("rc_all_to_all_v", [_vpp, _vpp, _i, ctypes.POINTER(ctypes.c_size_t), _i, _vp])
 _decl("rc_reserve_workspace", [_sz, _vp])
 _decl("rc_check_buffer", [_vp, _sz])
@@ -268,6 +277,64 @@ def rc_all_to_all_v(send: Sequence[Buf], recv: Sequence[Buf], counts, dtype=None
     arr = (ctypes.c_size_t * (p * p))(*flat)
     _check(lib.rc_all_to_all_v(_ptrs(send), _ptrs(recv), p, arr, _dt(dtype, send[0]), _stream(stream)),
            "rc_all_to_all_v")
+
+
+def rc_plan_buckets(numel: Sequence[int], elem_bytes: int, bucket_bytes: int):
+    """Bucket index of every tensor under the bucketer's rule (host only)."""
+    n = len(numel)
+    arr = (ctypes.c_size_t * max(1, n))(*[int(x) for x in numel])
+    out = (ctypes.c_int * max(1, n))()
+    nb = ctypes.c_int()
+    _check(lib.rc_plan_buckets(n, arr, elem_bytes, min(int(bucket_bytes), 2**64 - 1), out,
+                               ctypes.byref(nb)), "rc_plan_buckets")
+    return [out[i] for i in range(n)], nb.value
+
+
+class Bucketer:
+    """Gradient bucketing (rc_bucketer_*): p flat gradient buffers, tensors in
+    ready order; ready(t, stream) after tensor t's gradients are written on
+    every rank, flush(stream) at the end of the step."""
+
+    def __init__(self, flat: Sequence[Buf], numel: Sequence[int], bucket_bytes: int, dtype=None,
+                 scale=None, comm_stream=None):
+        p = len(flat)
+        self.numel = [int(x) for x in numel]
+        arr = (ctypes.c_size_t * len(numel))(*self.numel)
+        h = ctypes.c_void_p()
+        self._comm = comm_stream  # keep the stream object alive
+        _check(lib.rc_bucketer_create(ctypes.byref(h), _ptrs(flat), p, len(numel), arr,
+                                      min(int(bucket_bytes), 2**64 - 1), _dt(dtype, flat[0]),
+                                      1.0 / p if scale is None else scale, _stream(comm_stream)),
+               "rc_bucketer_create")
+        self.h = h.value
+
+    def buckets(self):
+        nb = ctypes.c_int()
+        _check(lib.rc_bucketer_num_buckets(self.h, ctypes.byref(nb)), "rc_bucketer_num_buckets")
+        out = []
+        for k in range(nb.value):
+            t0, t1, e0, ne = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t(), ctypes.c_size_t()
+            _check(lib.rc_bucketer_bucket(self.h, k, ctypes.byref(t0), ctypes.byref(t1), ctypes.byref(e0),
+                                          ctypes.byref(ne)), "rc_bucketer_bucket")
+            out.append((t0.value, t1.value, e0.value, ne.value))
+        return out
+
+    def ready(self, tensor: int, stream=None):
+        _check(lib.rc_bucketer_ready(self.h, tensor, _stream(stream)), "rc_bucketer_ready")
+
+    def flush(self, stream=None):
+        _check(lib.rc_bucketer_flush(self.h, _stream(stream)), "rc_bucketer_flush")
+
+    def close(self):
+        if self.h:
+            lib.rc_bucketer_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def rc_copy(src: Buf, dst: Buf, nbytes=None, stream=None):

@@ -26,6 +26,12 @@
  *         of N-1 steps (send one chunk to the next card, which accumulates);
  *         all-gather phase of N-1 steps (forward the finished chunk, receiver
  *         overwrites); 2(N-1) steps; card 0 ends the first phase holding chunk 0.
+ *  [DDP]  "分布式训练/推理", section "数据并行：切 batch，复制模型" -- naive DDP
+ *         all-reduces every gradient after backward (many calls, all exposed);
+ *         one flattened all-reduce saves calls but waits for the last gradient;
+ *         per-parameter hooks all-reduce each gradient as soon as it is ready
+ *         and hide communication under the rest of backward; measure the
+ *         communication left exposed after backward.
  *  [ZERO] "分布式训练/推理", section "显存账：不同数据并行的局限性" -- ZeRO-1
  *         shards the optimizer state (Adam moments, fp32 master weights) while
  *         every rank keeps full parameters; section "DDP 模型训练示例" -- the
@@ -226,6 +232,56 @@ rc_status rc_all_to_all_v(const void *const *send, void *const *recv, int p, con
  * recv[q][r*(n/p) + j] = send[r][q*(n/p) + j]. */
 rc_status rc_all_to_all(const void *const *send, void *const *recv, int p, size_t n, rc_dtype dt,
                         rc_stream_t stream);
+
+/*
+ * Gradient bucketing for data parallelism [DDP] -- a host-side runtime over
+ * rc_all_reduce; no kernels of its own.
+ *
+ * Every simulated rank keeps its gradients in one flat device buffer of
+ * sum(numel) elements of dt; tensor t occupies the same element range
+ * [off_t, off_t + numel[t]) of every rank's buffer, tensors in the order
+ * their gradients become ready.  Buckets are runs of consecutive whole
+ * tensors: a bucket takes tensors in order and closes as soon as it holds at
+ * least bucket_bytes (bucket_bytes = 0: one bucket per tensor; SIZE_MAX: one
+ * bucket for all).  A bucket is reduced by one in-place rc_all_reduce of its
+ * slice of every rank's buffer (op SUM, `scale`, e.g. 1/p for the average),
+ * so its fold order is that of an all-reduce of the slice.
+ */
+typedef struct rc_bucketer rc_bucketer;
+
+/* The bucket plan alone (host only, no GPU): bucket_of[t] receives tensor
+ * t's bucket index, *nbuckets the count.  elem_bytes > 0. */
+rc_status rc_plan_buckets(int ntensors, const size_t *numel, size_t elem_bytes, size_t bucket_bytes,
+                          int *bucket_of, int *nbuckets);
+
+/* Create a bucketer for p flat gradient buffers (device memory of the
+ * current device, each checked like rc_check_buffer).  The buffers and the
+ * communication stream `comm` must outlive the bucketer.  dt RC_INT32
+ * requires scale == 1. */
+rc_status rc_bucketer_create(rc_bucketer **out, void *const *flat, int p, int ntensors,
+                             const size_t *numel, size_t bucket_bytes, rc_dtype dt, float scale,
+                             rc_stream_t comm);
+
+/* Inspect the plan: the number of buckets, and bucket k's tensors
+ * [first_tensor, end_tensor) and element range (any output may be NULL). */
+rc_status rc_bucketer_num_buckets(const rc_bucketer *b, int *nbuckets);
+rc_status rc_bucketer_bucket(const rc_bucketer *b, int k, int *first_tensor, int *end_tensor,
+                             size_t *first_elem, size_t *nelem);
+
+/* Tensor t's gradients are complete on every rank in the order of stream
+ * `producer`: records an event there and makes `comm` wait for it; when t
+ * completes its bucket, enqueues the bucket's all-reduce on `comm`.  A tensor
+ * marked twice in one step returns RC_ERR_INVALID_ARG. */
+rc_status rc_bucketer_ready(rc_bucketer *b, int tensor, rc_stream_t producer);
+
+/* End of the step: `consumer` waits for every all-reduce enqueued so far and
+ * the bucketer resets for the next step.  RC_ERR_INVALID_ARG if a bucket was
+ * incomplete (a tensor never marked ready; that bucket was not reduced). */
+rc_status rc_bucketer_flush(rc_bucketer *b, rc_stream_t consumer);
+
+/* Release the bucketer's events and memory (NULL is a no-op).  Call it after
+ * the work it enqueued has been waited for. */
+rc_status rc_bucketer_destroy(rc_bucketer *b);
 
 /* AdamW hyperparameters of one optimizer step [ZERO]. */
 typedef struct rc_adamw_hparams {
