@@ -112,14 +112,14 @@ def special_values(p: int, n: int, seed: int, dt: str = "f32") -> List[np.ndarra
 
 
 def config(name: str):
-    """The five named workloads: a dict with everything needed to draw them."""
+    """The named workloads: a dict with everything needed to draw them."""
     cfgs = {
         "worked_example": dict(p=4, n=4, dt="f32", gen="worked"),
-        "cfg1": dict(p=4, n=65536, dt="f32", gen="uniform", seed=0),
-        "cfg2_ring": dict(p=8, n=2097152, dt="f32", gen="normal", seed=1, sigma=1e-2),
-        "cfg3_hier": dict(p=8, n=4194304, dt="bf16", gen="normal", seed=2, sigma=1.0, group=4),
-        "cfg4_params": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS // 8, dt="bf16", gen="uniform", seed=3),
-        "cfg4_grads": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS, dt="f32", gen="normal", seed=4, sigma=1e-3),
+        "uniform_p4_64k": dict(p=4, n=65536, dt="f32", gen="uniform", seed=0),
+        "ring_p8_2m_f32": dict(p=8, n=2097152, dt="f32", gen="normal", seed=1, sigma=1e-2),
+        "hier_2x4_4m_bf16": dict(p=8, n=4194304, dt="bf16", gen="normal", seed=2, sigma=1.0, group=4),
+        "llama_layer_param_shards_bf16": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS // 8, dt="bf16", gen="uniform", seed=3),
+        "llama_layer_grads_f32": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS, dt="f32", gen="normal", seed=4, sigma=1e-3),
         "zero1_state": dict(p=8, n=LLAMA2_7B_LAYER_ELEMS, gen="adam_state", seed=5),
     }
     return cfgs[name]

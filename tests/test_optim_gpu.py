@@ -143,7 +143,7 @@ def test_zero1_llama_layer_sampled(rc):
     p = 8
     N = rc_inputs.LLAMA2_7B_LAYER_ELEMS
     m = N // p
-    grads = rc_inputs.draw(rc_inputs.config("cfg4_grads"))
+    grads = rc_inputs.draw(rc_inputs.config("llama_layer_grads_f32"))
     master, ea, es = rc_inputs.draw(rc_inputs.config("zero1_state"))
     rng = np.random.default_rng(17)
     idx = np.unique(np.concatenate([

@@ -171,10 +171,10 @@ def test_ring_literal(rc, p, n, dt):
         check_canary(back, n * ESZ[dt])
 
 
-def test_cfg2_ring_and_oneshot_full_size(rc):
+def test_ring_and_oneshot_p8_8mib_full_size(rc):
     """8 ranks x 2,097,152 fp32 ~N(0, 1e-2), seed 1: literal 14-step ring and
     one-shot, both bit-identical to the oracle's ring simulation."""
-    cfg = rc_inputs.config("cfg2_ring")
+    cfg = rc_inputs.config("ring_p8_2m_f32")
     xs = rc_inputs.draw(cfg)
     p, n = cfg["p"], cfg["n"]
     want = oracle.ring_all_reduce(xs, "f32")
@@ -184,7 +184,7 @@ def test_cfg2_ring_and_oneshot_full_size(rc):
         rc.rc_ring_all_reduce(d, y, variant=variant)
         _sync(rc)
         for r in range(p):
-            assert_bits(to_host(y[r], "f32"), want[r], f"cfg2 {variant} r{r}")
+            assert_bits(to_host(y[r], "f32"), want[r], f"ring p8 8MiB {variant} r{r}")
         check_canary(back, n * 4)
 
 
@@ -219,11 +219,11 @@ def test_hier(rc, p, G, n, dt):
             check_canary(back, n * ESZ[dt])
 
 
-def test_cfg3_hier_full_size(rc):
+def test_hier_2x4_bf16_full_size(rc):
     """2 groups x 4 ranks, bf16 4,194,304 per rank ~N(0,1), seed 2: fused and
     staged bit-identical to the oracle's 3-phase simulation; within the fold
     bound (+1 bf16 ulp) of the flat all-reduce."""
-    cfg = rc_inputs.config("cfg3_hier")
+    cfg = rc_inputs.config("hier_2x4_4m_bf16")
     xs = rc_inputs.draw(cfg)
     p, n, G = cfg["p"], cfg["n"], cfg["group"]
     want = oracle.hier_all_reduce(xs, G, "bf16")
@@ -233,7 +233,7 @@ def test_cfg3_hier_full_size(rc):
         rc.rc_hier_all_reduce(d, y, G, variant=variant)
         _sync(rc)
         for r in range(p):
-            assert_bits(to_host(y[r], "bf16"), want[r], f"cfg3 {variant} r{r}")
+            assert_bits(to_host(y[r], "bf16"), want[r], f"hier 2x4 bf16 {variant} r{r}")
         check_canary(back, n * 2)
     flat, _ = empty_dev(n, "bf16", 1)
     rc.rc_reduce(d, flat[0])
@@ -245,7 +245,7 @@ def test_cfg3_hier_full_size(rc):
 
 
 # ------------------------------------------------------------ ZeRO-3 layer step
-def test_cfg4_zero3_layer(rc):
+def test_llama_layer_zero3_collectives(rc):
     """Llama-2-7B decoder layer (202,375,168 elements), 8 ranks: all_gather of
     bf16 parameter shards (compared in full), then reduce_scatter of fp32
     gradients ~N(0, 1e-3) with scale 1/8 to bf16 (sampled against the oracle,
@@ -253,18 +253,18 @@ def test_cfg4_zero3_layer(rc):
     p = 8
     N = rc_inputs.LLAMA2_7B_LAYER_ELEMS
     m = N // p
-    shards = rc_inputs.draw(rc_inputs.config("cfg4_params"))
+    shards = rc_inputs.draw(rc_inputs.config("llama_layer_param_shards_bf16"))
     d, _ = to_dev(shards, "bf16")
     full, _ = empty_dev(N, "bf16", p, pad_bytes=16)
     rc.rc_all_gather(d, full)
     _sync(rc)
     want = np.concatenate(shards)
     for r in range(p):
-        assert_bits(to_host(full[r], "bf16"), want, f"cfg4 all_gather r{r}")
+        assert_bits(to_host(full[r], "bf16"), want, f"llama layer all_gather r{r}")
     del full, d, want
     torch.cuda.empty_cache()
 
-    grads = rc_inputs.draw(rc_inputs.config("cfg4_grads"))
+    grads = rc_inputs.draw(rc_inputs.config("llama_layer_grads_f32"))
     g, _ = to_dev(grads, "f32")
     y, back = empty_dev(m, "bf16", p)
     rc.rc_reduce_scatter(g, y, in_dtype="f32", out_dtype="bf16", scale=1.0 / p)
@@ -276,7 +276,7 @@ def test_cfg4_zero3_layer(rc):
     ])).astype(np.uint64)
     ref = oracle.reduce_at(grads, idx, "f32", "bf16", "sum", 1.0 / p)
     got = np.concatenate([to_host(t, "bf16") for t in y])[idx.astype(np.int64)]
-    assert_bits(got, ref, "cfg4 reduce_scatter (sampled)")
+    assert_bits(got, ref, "llama layer reduce_scatter (sampled)")
     check_canary(back, m * 2)
 
 
