@@ -337,7 +337,7 @@ rc_status rc_zero1_step(const void *const *grads, void *const *params, float *co
 
 /*
  * Plain device copy dst[0, bytes) = src[0, bytes) with this library's
- * streaming kernel: the measured copy roofline the collectives are judged
+ * streaming kernel: the measured copy roofline the collectives are compared
  * against.  src and dst must not overlap.
  */
 rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream);
