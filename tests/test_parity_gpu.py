@@ -488,10 +488,14 @@ def test_register_path_matches_oracle(rc, dt, monkeypatch):
         assert_bits(np.concatenate([to_host(t, dt) for t in rs]), want[0], f"register rs {dt} {op}")
 
 
-@pytest.mark.parametrize("tile", ["4096", "16384"])
+@pytest.mark.parametrize("tile", ["4096", "16384", "register"])
 def test_fanout_tile_sizes(rc, tile, monkeypatch):
-    """The fan-out gives the same bytes whatever its tile size (ragged last tile)."""
-    monkeypatch.setenv("RC_FANOUT_TILE", tile)
+    """The fan-out gives the same bytes with the bulk-copy kernel at any tile
+    size and with the register kernel (ragged last tile)."""
+    if tile == "register":
+        monkeypatch.setenv("RC_FANOUT_REG", "1")
+    else:
+        monkeypatch.setenv("RC_FANOUT_TILE", tile)
     p, m = 8, 12345 * 8
     shards = rc_inputs.uniform(p, m, seed=12, dt="bf16")
     d, _ = to_dev(shards, "bf16")
