@@ -9,9 +9,7 @@ seed 1 (the ring / one-shot all-reduce workload), through
   all_gather (the bf16 shards), reduce (root 0), broadcast (root 0, in place),
   ring all_reduce (literal 14 steps), hierarchical all_reduce (2 x 4, fused).
 Timing: the whole step is captured once into a CUDA graph and the K steps
-replay it between one pair of CUDA events on the launching stream (the
-library launches its kernels with programmatic dependent launch, so inside
-the graph each kernel's launch overlaps the previous kernel's tail).  A split
+replay it between one pair of CUDA events on the launching stream.  A split
 per collective replays one graph per collective K more times, with an event
 between consecutive collectives (`--graph per_op` makes that the headline).
 Every collective of the step has its own inputs and outputs,
@@ -112,9 +110,9 @@ def step_ops(p=P, n=N):
 KERNEL_OF = {
     "all_reduce": ("rc_fold_tma_kernel", "fold.cu"),
     "reduce_scatter": ("rc_reduce_front_kernel", "reduce.cu"),
-    "all_gather": ("rc_fanout_bulk_kernel", "fanout.cu"),
+    "all_gather": ("rc_fanout_reg_kernel", "fanout.cu"),
     "reduce": ("rc_reduce_front_kernel", "reduce.cu"),
-    "broadcast": ("rc_fanout_bulk_kernel", "fanout.cu"),
+    "broadcast": ("rc_fanout_reg_kernel", "fanout.cu"),
     "ring_all_reduce": ("rc_ring_chain_kernel", "ring.cu"),
     "hier_all_reduce": ("rc_fold_tma_kernel", "fold.cu"),
 }
@@ -332,10 +330,7 @@ def run_ours(args):
     # graph (one host launch per collective instead of the binding's argument
     # marshalling and checks, which take longer than a collective on the GPU),
     # and the whole step once more into one graph.  The headline replays the
-    # step graph K times between one pair of events: inside it, every kernel
-    # is launched with programmatic dependent launch, so its launch and
-    # prologue overlap the previous kernel's tail (each kernel still waits for
-    # the previous one to finish before it touches memory).  The split per
+    # step graph K times between one pair of events.  The split per
     # collective replays the per-collective graphs K times with an event
     # before every collective and one after the last.
     for nm in names:
@@ -557,7 +552,7 @@ def run_ours(args):
                           "outputs, so between two reads of an op's inputs the other ops move > 500 MiB "
                           "(> 4x the 126 MB L2). " + (
                               "value: K replays of one CUDA graph of the whole step between one pair of "
-                              "CUDA events (kernels with programmatic dependent launch); per_op.us: K "
+                              "CUDA events; per_op.us: K "
                               "replays of one graph per collective, back to back, an event between "
                               "collectives" if step_graph is not None else
                               "value and per_op.us: K replays of one CUDA graph per collective, back to "

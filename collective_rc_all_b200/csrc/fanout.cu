@@ -1,5 +1,5 @@
-// fanout.cu -- all-gather and broadcast as a fan-out: a bulk-copy kernel
-// (default) and a register kernel.
+// fanout.cu -- all-gather and broadcast as a fan-out: a register kernel
+// (default) and a bulk-copy kernel.
 //
 // Pages: "分布式训练/推理", section "通信原语：rank、world size 和 collective
 // operations" (broadcast copies one rank's tensor to every rank; all-gather
@@ -207,13 +207,13 @@ cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s) {
   if (job.src_bytes == 0) return cudaSuccess;
   cudaError_t err;
   const int sms = device_sm_count();
-  // default: the bulk-copy kernel.  RC_FANOUT_REG=1 selects the register
-  // kernel, which is faster alone (7.6 vs 8.1 us for an 8 x 512 KiB bf16
-  // all-gather and 12.1 vs 12.4 us for an 8 MiB fp32 broadcast, each replayed
-  // back to back; 6.1 vs 5.5 TB/s on 64 MiB sources) but made a whole
-  // sequence of seven different collectives captured in one graph slower
-  // (139 vs 134 us per sequence, two runs each).
-  if (aligned && env_int("RC_FANOUT_REG", 0)) {
+  // default: the register kernel (faster alone: 7.6 vs 8.1 us for an
+  // 8 x 512 KiB bf16 all-gather and 12.1 vs 12.4 us for an 8 MiB fp32
+  // broadcast replayed back to back, 6.1 vs 5.5 TB/s on 64 MiB sources; and in
+  // a sequence of seven different collectives in one graph, 130-133 vs
+  // 133-134 us, with dependent launches off).  RC_FANOUT_BULK=1 selects the
+  // bulk-copy kernel.
+  if (aligned && !env_int("RC_FANOUT_BULK", 0)) {
     const uint64_t nv = job.src_bytes / 16;
     const uint64_t tps = (nv + kRegNT * kRegILP - 1) / (kRegNT * kRegILP);
     const uint64_t grid = tps * (uint64_t)job.nsrc;

@@ -1,6 +1,6 @@
 // launch.cuh -- how every kernel of this library is launched.
 //
-// Kernels go out with programmatic dependent launch: the launch carries the
+// Kernels can go out with programmatic dependent launch: the launch carries the
 // programmatic stream-serialization attribute, so the GPU may schedule the
 // kernel's thread blocks while the previous kernel in the stream is still
 // draining, and each kernel triggers its own dependents as soon as all of its
@@ -13,8 +13,13 @@
 // (shared-memory tables, mbarrier set-up) overlap the previous kernel's tail.
 // Stream capture turns the attribute into programmatic graph edges.
 //
-// RC_PDL=0 in the environment (read once per process) launches without the
-// attribute; griddepcontrol.wait then returns at once.
+// Off by default: RC_PDL=1 in the environment (read once per process) turns
+// it on.  Measured on a sequence of seven different collectives captured in
+// one graph, it changed nothing with the bulk-copy fan-out (133.8 vs 133.5 us)
+// and cost 5% with the register fan-out (138.8 vs 131.1 us), presumably
+// because the dependents' blocks, resident early and waiting at
+// griddepcontrol.wait, take issue slots from the running kernel.  Without
+// the attribute griddepcontrol.wait returns at once.
 #pragma once
 
 #include <cuda_runtime.h>

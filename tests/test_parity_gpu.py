@@ -492,9 +492,8 @@ def test_register_path_matches_oracle(rc, dt, monkeypatch):
 def test_fanout_tile_sizes(rc, tile, monkeypatch):
     """The fan-out gives the same bytes with the bulk-copy kernel at any tile
     size and with the register kernel (ragged last tile)."""
-    if tile == "register":
-        monkeypatch.setenv("RC_FANOUT_REG", "1")
-    else:
+    if tile != "register":
+        monkeypatch.setenv("RC_FANOUT_BULK", "1")
         monkeypatch.setenv("RC_FANOUT_TILE", tile)
     p, m = 8, 12345 * 8
     shards = rc_inputs.uniform(p, m, seed=12, dt="bf16")
