@@ -70,8 +70,7 @@ NCU_TRAFFIC = {
     "ring_all_reduce": {"bytes": 67128320 + 33989888, "src": "79d77f64a1dae252"},
     "all_reduce": {"bytes": 67130112 + 17357312, "src": "8395a3efc3921db4"},
     "reduce_scatter": {"bytes": 67121408 + 1258752, "src": "2bfc7ab651598460"},
-    "all_gather": {"bytes": 4205312 + 196096, "src": "7c1e06d78d330fd4"},
-}
+    "all_gather": {"bytes": 4201728 + 137472, "src": "a8c217689c27bb33"},
 
 
 def busbw_all_reduce(size_bytes: float, p: int, t: float) -> float:
