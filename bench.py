@@ -71,6 +71,7 @@ NCU_TRAFFIC = {
     "all_reduce": {"bytes": 67130112 + 17357312, "src": "8395a3efc3921db4"},
     "reduce_scatter": {"bytes": 67121408 + 1258752, "src": "2bfc7ab651598460"},
     "all_gather": {"bytes": 4201728 + 137472, "src": "a8c217689c27bb33"},
+}
 
 
 def busbw_all_reduce(size_bytes: float, p: int, t: float) -> float:
