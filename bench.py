@@ -460,41 +460,75 @@ def run_ours(args):
     if args.no_e2e:
         e2e_k = 0
 
-    # end to end: one set of inputs copied in from the host, every collective
-    # of the step on it, one copy of every result copied back
-    e2e_calls = {
-        "all_reduce": lambda: rc.rc_all_reduce(send, y_ar),
-        "reduce_scatter": lambda: rc.rc_reduce_scatter(send, y_rs, out_dtype="bf16", scale=1.0 / P),
-        "all_gather": lambda: rc.rc_all_gather(y_rs, y_ag),
-        "reduce": lambda: rc.rc_reduce(send, y_red, root=0),
-        "broadcast": lambda: rc.rc_broadcast(send[0], [send[0]] + y_bc[1:], root=0),
-        "ring_all_reduce": lambda: rc.rc_ring_all_reduce(send, y_ring, variant="literal"),
-        "hier_all_reduce": lambda: rc.rc_hier_all_reduce(send, y_hier, 4, variant="fused"),
-    }
+    # end to end: every step copies one set of inputs in from pinned host
+    # memory, runs every collective of the step on it through the Python API,
+    # and copies one copy of every result back.  PCIe is full duplex, so the
+    # steps are pipelined: inputs are double-buffered on the device, the
+    # host->device copy of step k+1 runs on its own stream while the
+    # device->host copy of step k runs on another; step k+1's collectives wait
+    # for its inputs and for the read-back of step k's results (which they
+    # overwrite).
+    send2 = [torch.empty_like(t) for t in send]
+    bufs = [send, send2]
 
-    def e2e_step():
-        for d, h in zip(send, host_in):
-            d.copy_(h, non_blocking=True)
+    def e2e_calls(buf):
+        return {
+            "all_reduce": lambda: rc.rc_all_reduce(buf, y_ar),
+            "reduce_scatter": lambda: rc.rc_reduce_scatter(buf, y_rs, out_dtype="bf16", scale=1.0 / P),
+            "all_gather": lambda: rc.rc_all_gather(y_rs, y_ag),
+            "reduce": lambda: rc.rc_reduce(buf, y_red, root=0),
+            "broadcast": lambda: rc.rc_broadcast(buf[0], [buf[0]] + y_bc[1:], root=0),
+            "ring_all_reduce": lambda: rc.rc_ring_all_reduce(buf, y_ring, variant="literal"),
+            "hier_all_reduce": lambda: rc.rc_hier_all_reduce(buf, y_hier, 4, variant="fused"),
+        }
+
+    calls_of = [e2e_calls(bufs[0]), e2e_calls(bufs[1])]
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event(), torch.cuda.Event()]     # inputs of buffer i landed
+    ev_used = [torch.cuda.Event(), torch.cuda.Event()]   # collectives done with buffer i
+    ev_out = torch.cuda.Event()                          # results of the last step read back
+    ev_used[0].record(stream)
+    ev_used[1].record(stream)
+    ev_out.record(stream)
+
+    def e2e_step(k):
+        i = k % 2
+        with torch.cuda.stream(h2d_s):
+            h2d_s.wait_event(ev_used[i])   # the step two back has finished reading buffer i
+            for d, h in zip(bufs[i], host_in):
+                d.copy_(h, non_blocking=True)
+            ev_in[i].record(h2d_s)
+        stream.wait_event(ev_in[i])
+        stream.wait_event(ev_out)          # the previous results have been read back
         for nm in names:
-            e2e_calls[nm]()
-        for h, d in zip(host_out, flat_outs):
-            h.copy_(d, non_blocking=True)
+            calls_of[i][nm]()
+        ev_used[i].record(stream)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(ev_used[i])
+            for h, d in zip(host_out, flat_outs):
+                h.copy_(d, non_blocking=True)
+            ev_out.record(d2h_s)
 
     e2e = None
     if e2e_k:
-        for _ in range(2):
-            e2e_step()
+        for k in range(2):
+            e2e_step(k)
         torch.cuda.synchronize()
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ea.record(stream)
-        for _ in range(e2e_k):
-            e2e_step()
+        h2d_s.wait_event(ea)   # no copy of the timed steps starts before the clock
+        d2h_s.wait_event(ea)
+        for k in range(e2e_k):
+            e2e_step(k)
+        stream.wait_event(ev_out)
         eb.record(stream)
         eb.synchronize()
         e2e_s, e2e_bytes = reduce_over_ranks(ea.elapsed_time(eb) * 1e-3, step_bytes * e2e_k, world,
                                              device=dev)
         e2e = {"value": round(e2e_bytes / e2e_s / 1e9, 2), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "pipelined": "H2D of step k+1 on one stream overlaps D2H of step k on another "
+                            "(double-buffered device inputs)"}
 
     if world > 1:
         import torch.distributed as dist
