@@ -44,6 +44,11 @@ rc_status cuda_fail(cudaError_t e, const char *what) {
 }
 }  // namespace
 
+rc_status report_error(rc_status st, const char *msg) {
+  snprintf(t_last_error, sizeof t_last_error, "%s", msg);
+  return st;
+}
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;

@@ -80,23 +80,26 @@ extern "C" {
 rc_status rc_plan_buckets(int ntensors, const size_t *numel, size_t elem_bytes, size_t bucket_bytes,
                           int *bucket_of, int *nbuckets) {
   if (ntensors < 0 || (ntensors > 0 && (!numel || !bucket_of)) || !nbuckets || elem_bytes == 0)
-    return RC_ERR_INVALID_ARG;
+    return rc::report_error(RC_ERR_INVALID_ARG, "rc_plan_buckets: bad arguments");
   *nbuckets = rc::plan_buckets(ntensors, numel, elem_bytes, bucket_bytes, bucket_of);
   return RC_OK;
 }
 
 rc_status rc_bucketer_create(rc_bucketer **out, void *const *flat, int p, int ntensors, const size_t *numel,
                              size_t bucket_bytes, rc_dtype dt, float scale, rc_stream_t comm) {
-  if (!out) return RC_ERR_INVALID_ARG;
+  if (!out) return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_create: out is NULL");
   *out = nullptr;
-  if (p < 1 || p > rc::kMaxP || ntensors < 1 || !numel || !flat) return RC_ERR_INVALID_ARG;
-  if (dt != RC_FP32 && dt != RC_BF16 && dt != RC_INT32) return RC_ERR_INVALID_ARG;
-  if (dt == RC_INT32 && scale != 1.0f) return RC_ERR_INVALID_ARG;
+  if (p < 1 || p > rc::kMaxP || ntensors < 1 || !numel || !flat)
+    return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_create: bad p, tensor list or buffer array");
+  if (dt != RC_FP32 && dt != RC_BF16 && dt != RC_INT32)
+    return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_create: unknown dtype");
+  if (dt == RC_INT32 && scale != 1.0f)
+    return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_create: int32 requires scale 1");
   const size_t esz = dt == RC_BF16 ? 2 : 4;
   uint64_t total = 0;
   for (int t = 0; t < ntensors; ++t) total += numel[t];
   for (int r = 0; r < p; ++r) {
-    if (!flat[r]) return RC_ERR_INVALID_ARG;
+    if (!flat[r]) return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_create: a gradient buffer is NULL");
     rc_status st = rc_check_buffer(flat[r], total * esz);
     if (st != RC_OK) return st;
   }
@@ -134,21 +137,22 @@ rc_status rc_bucketer_create(rc_bucketer **out, void *const *flat, int p, int nt
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     rc_bucketer_destroy(b);
-    return RC_ERR_CUDA;
+    return rc::report_error(RC_ERR_CUDA, "rc_bucketer_create: event creation failed");
   }
   *out = b;
   return RC_OK;
 }
 
 rc_status rc_bucketer_num_buckets(const rc_bucketer *b, int *nbuckets) {
-  if (!b || !nbuckets) return RC_ERR_INVALID_ARG;
+  if (!b || !nbuckets) return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_num_buckets: NULL argument");
   *nbuckets = (int)b->t0.size();
   return RC_OK;
 }
 
 rc_status rc_bucketer_bucket(const rc_bucketer *b, int k, int *first_tensor, int *end_tensor,
                              size_t *first_elem, size_t *nelem) {
-  if (!b || k < 0 || k >= (int)b->t0.size()) return RC_ERR_INVALID_ARG;
+  if (!b || k < 0 || k >= (int)b->t0.size())
+    return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_bucket: no such bucket");
   const int t0 = b->t0[k], t1 = b->t1[k];
   if (first_tensor) *first_tensor = t0;
   if (end_tensor) *end_tensor = t1;
@@ -158,13 +162,15 @@ rc_status rc_bucketer_bucket(const rc_bucketer *b, int k, int *first_tensor, int
 }
 
 rc_status rc_bucketer_ready(rc_bucketer *b, int tensor, rc_stream_t producer) {
-  if (!b || tensor < 0 || tensor >= (int)b->off.size()) return RC_ERR_INVALID_ARG;
-  if (b->seen[tensor]) return RC_ERR_INVALID_ARG;  // marked twice in one step
+  if (!b || tensor < 0 || tensor >= (int)b->off.size())
+    return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_ready: no such tensor");
+  if (b->seen[tensor])
+    return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_ready: tensor marked ready twice in one step");
   cudaError_t e = cudaEventRecord(b->ready_ev[tensor], (cudaStream_t)producer);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(b->comm, b->ready_ev[tensor], 0);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
-    return RC_ERR_CUDA;
+    return rc::report_error(RC_ERR_CUDA, "rc_bucketer_ready: event record / stream wait failed");
   }
   b->seen[tensor] = 1;
   const int k = b->bucket_of[tensor];
@@ -180,7 +186,7 @@ rc_status rc_bucketer_ready(rc_bucketer *b, int tensor, rc_stream_t producer) {
 }
 
 rc_status rc_bucketer_flush(rc_bucketer *b, rc_stream_t consumer) {
-  if (!b) return RC_ERR_INVALID_ARG;
+  if (!b) return rc::report_error(RC_ERR_INVALID_ARG, "rc_bucketer_flush: NULL bucketer");
   bool complete = true;
   for (size_t k = 0; k < b->pending.size(); ++k) complete = complete && b->pending[k] == 0;
   cudaError_t e = cudaEventRecord(b->done, b->comm);
@@ -191,9 +197,11 @@ rc_status rc_bucketer_flush(rc_bucketer *b, rc_stream_t consumer) {
   b->launched = 0;
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
-    return RC_ERR_CUDA;
+    return rc::report_error(RC_ERR_CUDA, "rc_bucketer_flush: event record / stream wait failed");
   }
-  return complete ? RC_OK : RC_ERR_INVALID_ARG;
+  return complete ? RC_OK
+                  : rc::report_error(RC_ERR_INVALID_ARG,
+                                     "rc_bucketer_flush: a bucket was incomplete (a tensor never marked ready)");
 }
 
 rc_status rc_bucketer_destroy(rc_bucketer *b) {

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "rankcoll.h"
+
 namespace rc {
 
 constexpr int kMaxP = 16;
@@ -122,6 +124,9 @@ cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s);
 
 // Device-side bounded waits report here (fanout.cu).
 cudaError_t read_and_clear_wait_timeouts(unsigned int *count);
+
+// Record msg as this thread's rc_last_error() and return st (api.cu).
+rc_status report_error(rc_status st, const char *msg);
 
 // Helpers shared by the launchers (api.cu).
 int device_sm_count();        // SMs of the current device (cached)

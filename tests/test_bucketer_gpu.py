@@ -113,8 +113,10 @@ def test_incomplete_and_double_ready_are_errors(rc):
     b.ready(0)
     with pytest.raises(rc.RankCollError):
         b.ready(0)
+    assert "twice" in rc.rc_last_error()
     with pytest.raises(rc.RankCollError):
         b.flush()  # tensors 1.. were never marked
+    assert "incomplete" in rc.rc_last_error()
     # the next step starts clean
     for t in range(len(SIZES)):
         b.ready(t)

@@ -43,6 +43,7 @@ def test_plan_rejects_bad_arguments(rc):
     arr = (ctypes.c_size_t * 2)(1, 2)
     out = (ctypes.c_int * 2)()
     assert rc.lib.rc_plan_buckets(2, arr, 0, 64, out, ctypes.byref(nb)) == 1   # zero element size
+    assert "rc_plan_buckets" in rc.rc_last_error()
 
 
 def test_bucketer_create_rejects_host_memory(rc):
