@@ -1052,6 +1052,135 @@ def run_ddp(args):
     return 0
 
 
+def run_configs(args):
+    """Every named workload's calls, timed (one JSON line per call):
+      uniform p=4 x 65,536 fp32         all_reduce, reduce_scatter, all_gather
+      ring p=8 x 2,097,152 fp32         ring literal, ring one-shot, all_reduce
+      hierarchical 2x4 x 4,194,304 bf16 fused, staged, flat all_reduce
+      Llama-2-7B layer p=8              all_gather of bf16 shards, reduce_scatter
+                                        fp32 -> bf16 x 1/8
+    Each call alone after an L2 flush outside its events (median of reps),
+    and back to back: one CUDA graph of 4 calls on 4 separate input/output
+    sets (1 set for the layer, whose buffers dwarf L2), replayed; per call =
+    time / calls.  GB/s on the minimum-bytes basis."""
+    import torch
+    import collective_rc_all_b200 as rc
+    import rc_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peak, _ = measured_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    gen = torch.Generator(device=dev)
+    TT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+    def rand(n, dt, sigma=1.0):
+        return (torch.randn(n, generator=gen, device=dev) * sigma).to(TT[dt])
+
+    def iso(fn, reps=20):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            torch.sum(clean, dim=0, out=sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e-3)
+        return float(np.median(ts))
+
+    def b2b(fns, reps=20):
+        for f in fns:
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for f in fns:
+                f()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e-3 / (reps * len(fns))
+
+    def emit(workload, call, byt, t_iso, t_b2b):
+        row = {"workload": workload, "call": call, "min_bytes": byt,
+               "isolated_us": round(t_iso * 1e6, 2), "isolated_gbs": round(byt / t_iso / 1e9, 1),
+               "isolated_frac_of_measured_hbm": round(byt / t_iso / 1e9 / peak, 4),
+               "back_to_back_us": round(t_b2b * 1e6, 2), "back_to_back_gbs": round(byt / t_b2b / 1e9, 1),
+               "back_to_back_frac_of_measured_hbm": round(byt / t_b2b / 1e9 / peak, 4)}
+        print(json.dumps(row), flush=True)
+
+    def sets(k, make):
+        return [make() for _ in range(k)]
+
+    # uniform p=4 x 65,536 fp32
+    p, n = 4, 65536
+    gen.manual_seed(0)
+    S = sets(4, lambda: {"x": [rand(n, "f32") for _ in range(p)], "y": [torch.empty(n, device=dev) for _ in range(p)],
+                         "rs": [torch.empty(n // p, device=dev) for _ in range(p)]})
+    for call, mk, byt in (
+            ("all_reduce", lambda d: (lambda: rc.rc_all_reduce(d["x"], d["y"])), 2 * p * n * 4),
+            ("reduce_scatter", lambda d: (lambda: rc.rc_reduce_scatter(d["x"], d["rs"])), p * n * 4 + n * 4),
+            ("all_gather", lambda d: (lambda: rc.rc_all_gather(d["rs"], d["y"])), n * 4 + p * n * 4)):
+        emit("uniform p=4 x 65,536 fp32", call, byt, iso(mk(S[0]), 50), b2b([mk(d) for d in S]))
+    del S
+
+    # ring p=8 x 2,097,152 fp32 N(0, 1e-2)
+    p, n = 8, 2097152
+    gen.manual_seed(1)
+    S = sets(4, lambda: {"x": [rand(n, "f32", 1e-2) for _ in range(p)], "y": [torch.empty(n, device=dev) for _ in range(p)]})
+    for call, mk in (
+            ("ring_all_reduce literal", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="literal"))),
+            ("ring_all_reduce one-shot", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="oneshot"))),
+            ("all_reduce", lambda d: (lambda: rc.rc_all_reduce(d["x"], d["y"])))):
+        emit("ring p=8 x 2,097,152 fp32", call, 2 * p * n * 4, iso(mk(S[0])), b2b([mk(d) for d in S]))
+    del S
+
+    # hierarchical 2 x 4 x 4,194,304 bf16 N(0, 1)
+    p, n = 8, 4194304
+    gen.manual_seed(2)
+    S = sets(4, lambda: {"x": [rand(n, "bf16") for _ in range(p)],
+                         "y": [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(p)]})
+    for call, mk in (
+            ("hier_all_reduce fused", lambda d: (lambda: rc.rc_hier_all_reduce(d["x"], d["y"], 4, variant="fused"))),
+            ("hier_all_reduce staged", lambda d: (lambda: rc.rc_hier_all_reduce(d["x"], d["y"], 4, variant="staged"))),
+            ("all_reduce (flat)", lambda d: (lambda: rc.rc_all_reduce(d["x"], d["y"])))):
+        emit("hierarchical 2x4 x 4,194,304 bf16", call, 2 * p * n * 2, iso(mk(S[0])), b2b([mk(d) for d in S]))
+    del S
+    torch.cuda.empty_cache()
+
+    # Llama-2-7B decoder layer, p=8: all_gather of bf16 shards, reduce_scatter fp32 -> bf16 x 1/8
+    N = rc_inputs.LLAMA2_7B_LAYER_ELEMS
+    m = N // p
+    gen.manual_seed(3)
+    shards = [(torch.rand(m, generator=gen, device=dev) * 2 - 1).to(torch.bfloat16) for _ in range(p)]
+    full = [torch.empty(N, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+    f = lambda: rc.rc_all_gather(shards, full)
+    emit("Llama-2-7B layer p=8", "all_gather bf16", N * 2 + p * N * 2, iso(f, 5), b2b([f], 5))
+    del full
+    torch.cuda.empty_cache()
+    gen.manual_seed(4)
+    grads = [rand(N, "f32", 1e-3) for _ in range(p)]
+    out = [torch.empty(m, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+    f = lambda: rc.rc_reduce_scatter(grads, out, out_dtype="bf16", scale=1.0 / p)
+    emit("Llama-2-7B layer p=8", "reduce_scatter fp32->bf16 x1/8", p * N * 4 + N * 2, iso(f, 5), b2b([f], 5))
+    rc.rc_stream_status()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1078,6 +1207,8 @@ def main(argv=None):
     ap.add_argument("--a2a", action="store_true")
     # the DDP gradient-bucketing workload: one JSON line
     ap.add_argument("--ddp", action="store_true")
+    # every named workload's calls, timed: one JSON line per call
+    ap.add_argument("--configs", action="store_true")
     ap.add_argument("--ddp-tokens", type=int, default=1024, help="tokens per rank of the synthetic backward")
     ap.add_argument("--zero1-elems", type=int, default=202375168,
                     help="parameters of the ZeRO-1 workload (default: one Llama-2-7B decoder layer)")
@@ -1093,6 +1224,8 @@ def main(argv=None):
         return run_a2a(args)
     if args.ddp:
         return run_ddp(args)
+    if args.configs:
+        return run_configs(args)
     return run_ours(args)
 
 

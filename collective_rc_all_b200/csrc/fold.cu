@@ -108,8 +108,10 @@ __device__ __forceinline__ int fold_rank(int k, int cg, int cl, int G, int ng) {
 }
 
 // GROUPED = false: the flat fold (G = p), a plain left-to-right fold;
-// GROUPED = true: the hierarchical fold with group boundaries.
-template <int PMAX, class TI, class TO, int OP, bool GROUPED>
+// GROUPED = true: the hierarchical fold with group boundaries, at fold
+// positions that are multiples of G -- compile-time when GS > 0 (GS == G),
+// from run-time bit masks when GS == 0.
+template <int PMAX, class TI, class TO, int OP, bool GROUPED, int GS = 0>
 __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_constant__ FoldParams a) {
   using Acc = typename TI::Acc;
   constexpr int VEC = kVec<TI>;
@@ -228,15 +230,18 @@ __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_co
           if (q < p) {
             Acc x[VEC];
             unpack<TI>(lds128(col + (uint32_t)q * tile_bytes), x);
-            if ((first >> q) & 1u) {
+            const bool is_first = GS > 0 ? (q % (GS > 0 ? GS : 1) == 0) : (((first >> q) & 1u) != 0);
+            if (is_first) {
 #pragma unroll
               for (int e = 0; e < VEC; ++e) Sg[e] = x[e];
             } else {
 #pragma unroll
               for (int e = 0; e < VEC; ++e) Sg[e] = combine<OP>(Sg[e], x[e]);
             }
-            if ((lastm >> q) & 1u) {
-              if (q < G) {
+            const bool is_last = GS > 0 ? (q % (GS > 0 ? GS : 1) == (GS > 0 ? GS : 1) - 1)
+                                        : (((lastm >> q) & 1u) != 0);
+            if (is_last) {
+              if (GS > 0 ? q < GS : q < G) {
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) T[e] = Sg[e];
               } else {
@@ -326,13 +331,16 @@ cudaError_t run_fold(const FoldJob &job, cudaStream_t s) {
   a.stages = stages;
   const size_t smem = (size_t)stages * a.stage_bytes;
 
-  auto kern = job.G == job.p ? rc_fold_tma_kernel<PMAX, TI, TO, OP, false>
-                             : rc_fold_tma_kernel<PMAX, TI, TO, OP, true>;
-  static std::atomic<uint64_t> attr_set[2];  // [GROUPED], one bit per device
+  // flat, grouped with groups of 4 (compile-time boundaries), other groups
+  const int variant = job.G == job.p ? 0 : (job.G == 4 && PMAX >= 8 ? 1 : 2);
+  auto kern = variant == 0 ? rc_fold_tma_kernel<PMAX, TI, TO, OP, false>
+            : variant == 1 ? rc_fold_tma_kernel<PMAX, TI, TO, OP, true, 4>
+                           : rc_fold_tma_kernel<PMAX, TI, TO, OP, true, 0>;
+  static std::atomic<uint64_t> attr_set[3];  // [variant], one bit per device
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  std::atomic<uint64_t> &flag = attr_set[job.G == job.p ? 0 : 1];
+  std::atomic<uint64_t> &flag = attr_set[variant];
   if (!(flag.load() & (1ull << (dev & 63)))) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (err != cudaSuccess) return err;
