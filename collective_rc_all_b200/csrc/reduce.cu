@@ -10,8 +10,9 @@
 //
 // Design (HBM-bound: (p-1) adds per element, 0.1 flop/byte at p = 8):
 //  * One thread owns whole 16-byte vectors: it issues all p 128-bit loads of
-//    ILP vectors before folding, so each thread keeps p*ILP*16 bytes in
-//    flight (256 B at p = 8) with no shared memory and no barriers.
+//    its ILP vectors (1 by default) before folding, so each thread keeps
+//    p*ILP*16 bytes in flight (128 B at p = 8) with no shared memory and no
+//    barriers.
 //  * The fold order of element i depends only on its chunk c = i / C:
 //    ranks (c+1)%p, ..., c.  Vectors never straddle a chunk (C % VEC == 0 is
 //    required for the vector path), so the rotated rank list is computed once
@@ -25,6 +26,7 @@
 //  * Results are written once per destination with 16-byte stores (8-byte for
 //    an fp32 -> bf16 reduce-scatter).
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -227,16 +229,23 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
     return cudaSuccess;
   }
   if (vector) {
-    constexpr int ILP = PMAX <= 8 ? 2 : 1;
     a.nvec = n / VEC;
     if (a.nvec > 0) {
       const uint64_t cvec = C / VEC;
-      const uint64_t tpc = (cvec + kNT * ILP - 1) / (kNT * ILP);
-      const uint64_t grid = tpc * (uint64_t)p;
-      if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
-      if ((err = launch_kernel(rc_reduce_front_kernel<PMAX, TI, TO, OP, ILP>, dim3((unsigned)grid), dim3(kNT),
-                               0, s, a, tpc)) != cudaSuccess)
-        return err;
+      auto go = [&](auto ilp_tag) -> cudaError_t {
+        constexpr int ILP = decltype(ilp_tag)::value;
+        const uint64_t tpc = (cvec + kNT * ILP - 1) / (kNT * ILP);
+        const uint64_t grid = tpc * (uint64_t)p;
+        if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
+        return launch_kernel(rc_reduce_front_kernel<PMAX, TI, TO, OP, ILP>, dim3((unsigned)grid), dim3(kNT), 0,
+                             s, a, tpc);
+      };
+      // one vector per thread: 12.0 vs 12.3 us for the p = 8 x 8 MiB fp32 ->
+      // bf16 reduce-scatter replayed back to back (more blocks per SM, fewer
+      // registers); RC_FRONT_ILP=2 selects two
+      const int ilp = env_int("RC_FRONT_ILP", 1);
+      err = ilp == 1 ? go(std::integral_constant<int, 1>()) : go(std::integral_constant<int, 2>());
+      if (err != cudaSuccess) return err;
     }
     if (a.nvec * VEC < n) {
       if ((err = launch_kernel(rc_reduce_tail_kernel<PMAX, TI, TO, OP>, dim3(1), dim3(32), 0, s, a,
