@@ -68,8 +68,8 @@ NCU_TRAFFIC = {
     # op: DRAM bytes per launch (read + write, one cold-cache ncu launch of the
     # step's workload), kernel source hash at capture time
     "ring_all_reduce": {"bytes": 67128320 + 33989888, "src": "79d77f64a1dae252"},
-    "all_reduce": {"bytes": 67130112 + 17357312, "src": "8395a3efc3921db4"},
-    "reduce_scatter": {"bytes": 67121408 + 1258752, "src": "2bfc7ab651598460"},
+    "all_reduce": {"bytes": 67132416 + 17382912, "src": "4da48bcfd1ebc3c2"},
+    "reduce_scatter": {"bytes": 67119616 + 1202176, "src": "f117e77e7724cc8d"},
     "all_gather": {"bytes": 4201728 + 137472, "src": "a8c217689c27bb33"},
 }
 
