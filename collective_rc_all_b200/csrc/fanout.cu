@@ -7,7 +7,7 @@
 // "FSDP 的执行顺序" (parameter shards all-gathered before the module runs).
 //
 // Register kernel: every thread loads its 16-byte vectors of one source once
-// and stores them to each destination (one block per 16 KiB of a source, the
+// and stores them to each destination (one block per 8 KiB of a source, the
 // blocks sweeping the sources as a front).
 //
 // Bulk-copy kernel: each source tile is read from HBM ONCE into the CTA's own shared memory by
@@ -24,6 +24,7 @@
 // and returns; rc_stream_status() reports RC_ERR_TIMEOUT.
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 
 #include "bulk.cuh"
 #include "common.cuh"
@@ -125,8 +126,8 @@ __global__ void __launch_bounds__(32) rc_fanout_bulk_kernel(const __grid_constan
 // once and stores them to each destination rank.  Blocks sweep the sources as
 // a front.
 constexpr int kRegNT = 256;
-constexpr int kRegILP = 4;
 
+template <int kRegILP>
 __global__ void __launch_bounds__(kRegNT) rc_fanout_reg_kernel(const __grid_constant__ FanoutParams a,
                                                                uint64_t tiles_per_src) {
   pdl_wait();
@@ -215,10 +216,20 @@ cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s) {
   // bulk-copy kernel.
   if (aligned && !env_int("RC_FANOUT_BULK", 0)) {
     const uint64_t nv = job.src_bytes / 16;
-    const uint64_t tps = (nv + kRegNT * kRegILP - 1) / (kRegNT * kRegILP);
-    const uint64_t grid = tps * (uint64_t)job.nsrc;
-    if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
-    return launch_kernel(rc_fanout_reg_kernel, dim3((unsigned)grid), dim3(kRegNT), 0, s, a, tps);
+    auto go = [&](auto ilp_tag) -> cudaError_t {
+      constexpr int ILP = decltype(ilp_tag)::value;
+      const uint64_t tps = (nv + kRegNT * ILP - 1) / (kRegNT * ILP);
+      const uint64_t grid = tps * (uint64_t)job.nsrc;
+      if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
+      return launch_kernel(rc_fanout_reg_kernel<ILP>, dim3((unsigned)grid), dim3(kRegNT), 0, s, a, tps);
+    };
+    // vectors per thread: 2 measured best in the one-graph sequence of seven
+    // collectives (131.0 us against 131.5 for 1 and 132.0 for 4); alone, the
+    // all-gather prefers 4 (7.9 vs 8.2 us) and the broadcast 2 (12.4 vs 12.6)
+    const int ilp = env_int("RC_FANOUT_ILP", 2);
+    if (ilp == 1) return go(std::integral_constant<int, 1>());
+    if (ilp == 2) return go(std::integral_constant<int, 2>());
+    return go(std::integral_constant<int, 4>());
   }
   if (aligned) {
     // tile: the largest power of two <= 32 KiB that still gives every SM about
