@@ -70,7 +70,7 @@ NCU_TRAFFIC = {
     "ring_all_reduce": {"bytes": 67128320 + 33989888, "src": "79d77f64a1dae252"},
     "all_reduce": {"bytes": 67132416 + 17382912, "src": "4da48bcfd1ebc3c2"},
     "reduce_scatter": {"bytes": 67119616 + 1202176, "src": "f117e77e7724cc8d"},
-    "all_gather": {"bytes": 4201728 + 137472, "src": "a8c217689c27bb33"},
+    "all_gather": {"bytes": 4200448 + 162048, "src": "222781d7ad9587f7"},
 }
 
 
@@ -294,12 +294,30 @@ def run_ours(args):
     own = lambda: [t.clone() for t in send]
     f32 = lambda k: [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(k)]
     bf16 = lambda k, n: [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(k)]
-    s_ar, s_rs, s_red, s_bc, s_ring, s_hier = own(), own(), own(), own(), own(), own()
-    y_ar, y_ring, y_hier = f32(P), f32(P), f32(P)
-    y_rs, ag_in, y_ag = bf16(P, m), bf16(P, m), bf16(P, N)
-    y_red = torch.empty(N, dtype=torch.float32, device=dev)
-    y_bc = [s_bc[0]] + f32(P - 1)          # root 0 in place
-    rc.rc_reduce_scatter(send, ag_in, out_dtype="bf16", scale=1.0 / P)  # the all-gather's shards
+    def buffer_set():
+        """Inputs (copies of the step's inputs) and outputs of every collective."""
+        B = {"s_ar": own(), "s_rs": own(), "s_red": own(), "s_bc": own(), "s_ring": own(), "s_hier": own(),
+             "y_ar": f32(P), "y_ring": f32(P), "y_hier": f32(P),
+             "y_rs": bf16(P, m), "ag_in": bf16(P, m), "y_ag": bf16(P, N),
+             "y_red": torch.empty(N, dtype=torch.float32, device=dev)}
+        B["y_bc"] = [B["s_bc"][0]] + f32(P - 1)          # root 0 in place
+        rc.rc_reduce_scatter(send, B["ag_in"], out_dtype="bf16", scale=1.0 / P)  # the all-gather's shards
+        return B
+
+    def calls_of(B):
+        return {
+            "all_reduce": lambda: rc.rc_all_reduce(B["s_ar"], B["y_ar"]),
+            "reduce_scatter": lambda: rc.rc_reduce_scatter(B["s_rs"], B["y_rs"], out_dtype="bf16", scale=1.0 / P),
+            "all_gather": lambda: rc.rc_all_gather(B["ag_in"], B["y_ag"]),
+            "reduce": lambda: rc.rc_reduce(B["s_red"], B["y_red"], root=0),
+            "broadcast": lambda: rc.rc_broadcast(B["s_bc"][0], B["y_bc"], root=0),
+            "ring_all_reduce": lambda: rc.rc_ring_all_reduce(B["s_ring"], B["y_ring"], variant="literal"),
+            "hier_all_reduce": lambda: rc.rc_hier_all_reduce(B["s_hier"], B["y_hier"], 4, variant="fused"),
+        }
+
+    B0 = buffer_set()
+    y_ar, y_rs, y_ag, y_red, y_bc, y_ring, y_hier = (B0[k] for k in ("y_ar", "y_rs", "y_ag", "y_red", "y_bc",
+                                                                     "y_ring", "y_hier"))
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -308,15 +326,7 @@ def run_ours(args):
         flush.zero_()
         torch.sum(clean, dim=0, out=sink)
 
-    calls = {
-        "all_reduce": lambda: rc.rc_all_reduce(s_ar, y_ar),
-        "reduce_scatter": lambda: rc.rc_reduce_scatter(s_rs, y_rs, out_dtype="bf16", scale=1.0 / P),
-        "all_gather": lambda: rc.rc_all_gather(ag_in, y_ag),
-        "reduce": lambda: rc.rc_reduce(s_red, y_red, root=0),
-        "broadcast": lambda: rc.rc_broadcast(s_bc[0], y_bc, root=0),
-        "ring_all_reduce": lambda: rc.rc_ring_all_reduce(s_ring, y_ring, variant="literal"),
-        "hier_all_reduce": lambda: rc.rc_hier_all_reduce(s_hier, y_hier, 4, variant="fused"),
-    }
+    calls = calls_of(B0)
     if args.ops:
         keep = args.ops.split(",")
         unknown = set(keep) - set(calls)
@@ -416,6 +426,33 @@ def run_ours(args):
     # this library's kernels inside the headline's timed region: the kernels
     # the captured graph(s) hold, times the replays
     launches = K * launches_per_step
+    # each collective back to back with itself: one graph of 4 calls of it
+    # on 4 separate input/output sets (4 x its footprint > L2), replayed K
+    # times -- its throughput as a stream of calls, every write-back paid
+    rep_sets = [B0] + [buffer_set() for _ in range(3)]
+    torch.cuda.synchronize()
+    rep_s = {}
+    for nm in names:
+        fs = [calls_of(Bx)[nm] for Bx in rep_sets]
+        for f in fs:
+            f()   # one-time set-up outside capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for f in fs:
+                f()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+        rep_s[nm] = a.elapsed_time(b) * 1e-3 / (K * len(fs))
+        del g
+    del rep_sets
     time.sleep(0.3)
     clk = clocks.stop()
     if world > 1:
@@ -551,6 +588,8 @@ def run_ours(args):
                       "gbs": round(b / t / 1e9, 1),
                       "frac_of_measured_hbm": round(b / t / 1e9 / peak, 4),
                       "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4) if copy_gbs else None,
+                      "repeated_us": round(rep_s[nm] * 1e6, 2),
+                      "repeated_frac_of_measured_hbm": round(b / rep_s[nm] / 1e9 / peak, 4),
                       "isolated_us": round(ti * 1e6, 2),
                       "isolated_frac_of_measured_hbm": round(b / ti / 1e9 / peak, 4)}
     if "all_reduce" in per_op:
@@ -591,7 +630,9 @@ def run_ours(args):
                               "collectives" if step_graph is not None else
                               "value and per_op.us: K replays of one CUDA graph per collective, back to "
                               "back, an event between collectives") +
-                          ". per_op.isolated_*: each collective alone (plain call) after a 512 MiB "
+                          ". per_op.repeated_*: one graph of 4 calls of the collective on 4 separate "
+                          "input/output sets, replayed K times. per_op.isolated_*: each collective alone (plain "
+                          "call) after a 512 MiB "
                           "write + 256 MiB read L2 flush outside its events"),
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": kname, "op": dom,
