@@ -1097,6 +1097,7 @@ def run_configs(args):
     """Every named workload's calls, timed (one JSON line per call):
       uniform p=4 x 65,536 fp32         all_reduce, reduce_scatter, all_gather
       ring p=8 x 2,097,152 fp32         ring literal, ring one-shot, all_reduce
+      ring p=8 x 2,097,152 bf16         ring literal (workspace), no-allocation ring, one-shot
       hierarchical 2x4 x 4,194,304 bf16 fused, staged, flat all_reduce
       Llama-2-7B layer p=8              all_gather of bf16 shards, reduce_scatter
                                         fp32 -> bf16 x 1/8
@@ -1188,6 +1189,21 @@ def run_configs(args):
             ("ring_all_reduce one-shot", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="oneshot"))),
             ("all_reduce", lambda d: (lambda: rc.rc_all_reduce(d["x"], d["y"])))):
         emit("ring p=8 x 2,097,152 fp32", call, 2 * p * n * 4, iso(mk(S[0])), b2b([mk(d) for d in S]))
+    del S
+
+    # ring p=8 x 2,097,152 bf16 (4 MiB per rank): fp32 partials in the
+    # library workspace, or in the fixed scratch of the no-allocation entry
+    # point (2 x 8 x 262,144 floats, exactly its 16 MiB)
+    p, n = 8, 2097152
+    gen.manual_seed(1)
+    S = sets(4, lambda: {"x": [rand(n, "bf16", 1e-2) for _ in range(p)],
+                         "y": [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(p)]})
+    rc.rc_reserve_workspace(2 * p * (n // p) * 4)
+    for call, mk in (
+            ("ring_all_reduce literal (workspace)", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="literal"))),
+            ("ring_all_reduce_noalloc", lambda d: (lambda: rc.rc_ring_all_reduce_noalloc(d["x"], d["y"]))),
+            ("ring_all_reduce one-shot", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="oneshot")))):
+        emit("ring p=8 x 2,097,152 bf16", call, 2 * p * n * 2, iso(mk(S[0])), b2b([mk(d) for d in S]))
     del S
 
     # hierarchical 2 x 4 x 4,194,304 bf16 N(0, 1)
