@@ -108,13 +108,13 @@ def step_ops(p=P, n=N):
 
 
 KERNEL_OF = {
-    "all_reduce": ("rc_fold_tma_kernel", "fold.cu"),
+    "all_reduce": ("rc_reduce_front_kernel", "reduce.cu"),
     "reduce_scatter": ("rc_reduce_front_kernel", "reduce.cu"),
     "all_gather": ("rc_fanout_reg_kernel", "fanout.cu"),
     "reduce": ("rc_reduce_front_kernel", "reduce.cu"),
     "broadcast": ("rc_fanout_reg_kernel", "fanout.cu"),
     "ring_all_reduce": ("rc_ring_chain_kernel", "ring.cu"),
-    "hier_all_reduce": ("rc_fold_tma_kernel", "fold.cu"),
+    "hier_all_reduce": ("rc_hier_front_kernel", "hier.cu"),
 }
 
 

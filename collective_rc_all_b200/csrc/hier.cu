@@ -115,6 +115,124 @@ __global__ void __launch_bounds__(kNT) rc_hier_reg_kernel(const __grid_constant_
   }
 }
 
+// Front kernel (default fused path): one 256-thread block per 256 vectors of
+// one segment, the segments being the runs of S = min(CG, CL) elements on
+// which both chunk indices are constant (used when the larger chunk length is
+// a multiple of the smaller, as for every p and G that divide n evenly).
+// Each thread loads the p vectors of its offset in the segment's fold order
+// -- position k = t*GS + j is rank ((cl+1+t) mod ng)*GS + (cg+1+j) mod GS --
+// folds each group of GS, then the group results, and writes the result to
+// every rank.  Group size compile-time (GS), so the boundaries cost nothing.
+template <int PMAX, class T, int OP, int GS>
+__global__ void __launch_bounds__(kNT) rc_hier_front_kernel(const __grid_constant__ HierParams a,
+                                                            uint64_t seg_vecs, uint64_t tiles_per_seg) {
+  using Acc = typename T::Acc;
+  constexpr int VEC = kVec<T>;
+  pdl_wait();
+  pdl_trigger();
+  const int p = a.p, ng = a.ng;
+  const uint64_t sg = blockIdx.x / tiles_per_seg;
+  const uint64_t v0 = sg * seg_vecs + (blockIdx.x - sg * tiles_per_seg) * (uint64_t)kNT;
+  const uint64_t vend0 = (sg + 1) * seg_vecs, nv = a.n / VEC;
+  const uint64_t vend = vend0 < nv ? vend0 : nv;
+  const uint64_t v = v0 + threadIdx.x;
+  if (v >= vend) return;
+  const uint64_t e0 = sg * seg_vecs * VEC;  // first element of the segment
+  const int cg = (int)(e0 / a.CG), cl = (int)(e0 / a.CL);
+  uint4 raw[PMAX];
+#pragma unroll
+  for (int k = 0; k < PMAX; ++k) {
+    if (k < p) {
+      const int t = k / GS, j = k - t * GS;
+      int gg = cl + 1 + t;
+      while (gg >= ng) gg -= ng;
+      int m = cg + 1 + j;
+      while (m >= GS) m -= GS;
+      raw[k] = ld_stream_v4(a.x[gg * GS + m] + v * 16);
+    }
+  }
+  Acc tot[VEC], grp[VEC];
+#pragma unroll
+  for (int k = 0; k < PMAX; ++k) {
+    if (k < p) {
+      Acc x[VEC];
+      unpack<T>(raw[k], x);
+      if (k % GS == 0) {
+#pragma unroll
+        for (int q = 0; q < VEC; ++q) grp[q] = x[q];
+      } else {
+#pragma unroll
+        for (int q = 0; q < VEC; ++q) grp[q] = combine<OP>(grp[q], x[q]);
+      }
+      if (k % GS == GS - 1) {
+        if (k < GS) {
+#pragma unroll
+          for (int q = 0; q < VEC; ++q) tot[q] = grp[q];
+        } else {
+#pragma unroll
+          for (int q = 0; q < VEC; ++q) tot[q] = combine<OP>(tot[q], grp[q]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < VEC; ++q) tot[q] = finish<OP>(tot[q], a.scale);
+  const uint64_t off = v * VEC * (uint64_t)T::kBytes;
+#pragma unroll
+  for (int r = 0; r < PMAX; ++r)
+    if (r < p) store_vec<T, VEC>(a.y[r] + off, tot);
+}
+
+template <int PMAX, class T, int OP>
+cudaError_t try_front(const HierJob &job, cudaStream_t s, bool *done) {
+  *done = false;
+  constexpr int VEC = kVec<T>;
+  HierParams a{};
+  a.p = job.p;
+  a.G = job.G;
+  a.ng = job.p / job.G;
+  a.n = job.n;
+  a.CG = (job.n + a.G - 1) / a.G;
+  a.CL = (job.n + a.ng - 1) / a.ng;
+  a.scale = job.scale;
+  bool ok = a.n % VEC == 0 && a.CG % VEC == 0 && a.CL % VEC == 0;
+  for (int r = 0; r < job.p; ++r) {
+    a.x[r] = static_cast<const char *>(job.x[r]);
+    a.y[r] = static_cast<char *>(job.y[r]);
+    ok = ok && reinterpret_cast<uintptr_t>(job.x[r]) % 16 == 0 && reinterpret_cast<uintptr_t>(job.y[r]) % 16 == 0;
+  }
+  const uint64_t S = std::min(a.CG, a.CL), Lg = std::max(a.CG, a.CL);
+  ok = ok && S > 0 && Lg % S == 0 && (job.G == 2 || job.G == 4 || job.G == 8);
+  if (!ok) return cudaSuccess;
+  const uint64_t seg_vecs = S / VEC;
+  const uint64_t nseg = (a.n / VEC + seg_vecs - 1) / seg_vecs;
+  const uint64_t tps = (seg_vecs + kNT - 1) / kNT;
+  const uint64_t grid = nseg * tps;
+  if (grid == 0 || grid > 0x7fffffffull) return cudaSuccess;
+  *done = true;
+  if (job.G == 2) return launch_kernel(rc_hier_front_kernel<PMAX, T, OP, 2>, dim3((unsigned)grid), dim3(kNT), 0, s, a, seg_vecs, tps);
+  if (job.G == 4) return launch_kernel(rc_hier_front_kernel<PMAX, T, OP, 4>, dim3((unsigned)grid), dim3(kNT), 0, s, a, seg_vecs, tps);
+  return launch_kernel(rc_hier_front_kernel<PMAX, T, OP, 8>, dim3((unsigned)grid), dim3(kNT), 0, s, a, seg_vecs, tps);
+}
+
+template <class T, int OP>
+cudaError_t front_by_p(const HierJob &job, cudaStream_t s, bool *done) {
+  if (job.p <= 4) return try_front<4, T, OP>(job, s, done);
+  if (job.p <= 8) return try_front<8, T, OP>(job, s, done);
+  return try_front<16, T, OP>(job, s, done);
+}
+
+template <class T>
+cudaError_t front_by_op(const HierJob &job, cudaStream_t s, bool *done) {
+  switch (job.op) {
+    case kSum: return front_by_p<T, kSum>(job, s, done);
+    case kMax: return front_by_p<T, kMax>(job, s, done);
+    case kMin: return front_by_p<T, kMin>(job, s, done);
+  }
+  *done = false;
+  return cudaSuccess;
+}
+
 template <int PMAX, class T, int OP>
 cudaError_t run_fused(const HierJob &job, cudaStream_t s) {
   HierParams a{};
@@ -179,6 +297,18 @@ cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s) {
   for (int r = 0; r < job.p; ++r) {
     f.src[r] = job.x[r];
     f.dst[r] = job.y[r];
+  }
+  // default: the register front kernel; RC_HIER_FOLD=1 selects the
+  // shared-memory-staged fold (both give the same bits)
+  if (!env_int("RC_HIER_FOLD", 0)) {
+    bool done = false;
+    cudaError_t err = cudaSuccess;
+    switch (job.dt) {
+      case kF32: err = front_by_op<F32>(job, s, &done); break;
+      case kBF16: err = front_by_op<BF16>(job, s, &done); break;
+      case kI32: err = front_by_op<I32>(job, s, &done); break;
+    }
+    if (done || err != cudaSuccess) return err;
   }
   if (fold_tma_eligible(f)) return launch_fold_tma(f, s);
   switch (job.dt) {

@@ -217,7 +217,11 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
   f.ndst = a.ndst;
   for (int r = 0; r < p; ++r) f.src[r] = job.src[r];
   for (int r = 0; r < ndst; ++r) f.dst[r] = job.dst[r];
-  if (vector && job.mode == kModeAll && fold_tma_eligible(f)) {
+  // The shared-memory-staged fold is the all-reduce's alternative path
+  // (RC_AR_FOLD=1): with one vector per thread the register front kernel
+  // measured faster for the p = 8 x 8 MiB fp32 all-reduce (23.4 vs 25.3 us
+  // back to back, 20.5 vs 23.6 us alone).
+  if (vector && job.mode == kModeAll && env_int("RC_AR_FOLD", 0) && fold_tma_eligible(f)) {
     // the staged fold covers whole vectors; the tail (n % VEC elements) is scalar
     if ((err = launch_fold_tma(f, s)) != cudaSuccess) return err;
     a.nvec = n / VEC;

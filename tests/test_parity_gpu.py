@@ -518,3 +518,28 @@ def test_copy_kernel(rc, nbytes):
     _sync(rc)
     assert torch.equal(a, b[:nbytes])
     assert int(b[nbytes:].sum()) == 0
+
+
+@pytest.mark.parametrize("dt", DTS)
+@pytest.mark.parametrize("p,G", [(8, 4), (8, 2), (16, 4), (4, 2)])
+def test_staged_fold_paths_match_oracle(rc, dt, p, G, monkeypatch):
+    """The shared-memory-staged fold, the alternative path of the all-reduce
+    (RC_AR_FOLD=1) and of the fused hierarchical all-reduce (RC_HIER_FOLD=1),
+    gives the oracle's bits too (ragged tail included)."""
+    monkeypatch.setenv("RC_AR_FOLD", "1")
+    monkeypatch.setenv("RC_HIER_FOLD", "1")
+    n = p * 4096 + p * 24 + (8 if dt != "bf16" else 16)
+    xs = _data(p, n, dt, seed=41 + p + G)
+    d, _ = to_dev(xs, dt)
+    for op in OPS:
+        y, back = empty_dev(n, dt, p)
+        rc.rc_all_reduce(d, y, op=op)
+        h, _ = empty_dev(n, dt, p)
+        rc.rc_hier_all_reduce(d, h, G, op=op)
+        _sync(rc)
+        want = oracle.all_reduce(xs, dt, op)
+        want_h = oracle.hier_all_reduce(xs, G, dt, op)
+        for r in (0, p - 1):
+            assert_bits(to_host(y[r], dt), want[r], f"staged fold all_reduce {dt} {op}")
+            assert_bits(to_host(h[r], dt), want_h[r], f"staged fold hier {dt} {op} G={G}")
+        check_canary(back, n * (2 if dt == "bf16" else 4))
