@@ -68,9 +68,10 @@ NCU_TRAFFIC = {
     # op: DRAM bytes per launch (read + write, one cold-cache ncu launch of the
     # step's workload), kernel source hash at capture time
     "ring_all_reduce": {"bytes": 67128320 + 33989888, "src": "79d77f64a1dae252"},
-    "all_reduce": {"bytes": 67132416 + 17382912, "src": "4da48bcfd1ebc3c2"},
-    "reduce_scatter": {"bytes": 67119616 + 1202176, "src": "f117e77e7724cc8d"},
+    "all_reduce": {"bytes": 67120640 + 13718528, "src": "1ed4bd8024e65e84"},
+    "reduce_scatter": {"bytes": 67119104 + 1223680, "src": "1ed4bd8024e65e84"},
     "all_gather": {"bytes": 4200448 + 162048, "src": "222781d7ad9587f7"},
+    "hier_all_reduce": {"bytes": 67121408 + 14397184, "src": "c29ec89dde043b30"},
 }
 
 
