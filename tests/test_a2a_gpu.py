@@ -145,3 +145,13 @@ def test_overlapping_send_and_recv_rejected(rc):
     with pytest.raises(rc.RankCollError):
         rc.rc_all_to_all(send, [other[0]] * p)  # receivers overlap one another
     assert rc.rc_launch_count() == before
+
+
+def test_single_rank_is_a_copy(rc):
+    xs = _data(1, 1000, "f32", 77)
+    d, _ = to_dev(xs, "f32")
+    y, back = empty_dev(1000, "f32", 1)
+    rc.rc_all_to_all(d, y)
+    _sync(rc)
+    assert_bits(to_host(y[0], "f32"), xs[0], "a2a p=1")
+    check_canary(back, 4000)

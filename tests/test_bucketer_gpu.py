@@ -124,3 +124,17 @@ def test_incomplete_and_double_ready_are_errors(rc):
     torch.cuda.synchronize()
     rc.rc_stream_status()
     b.close()
+
+
+def test_single_rank_bucketer(rc):
+    """p = 1: every bucket's all-reduce is the identity times scale (1)."""
+    host = rc_inputs.uniform(1, sum(SIZES), seed=8, dt="f32")
+    flat = _flat(host, "f32")
+    b = rc.Bucketer(flat, SIZES, 16 << 10, scale=1.0)
+    for t in range(len(SIZES)):
+        b.ready(t)
+    b.flush()
+    torch.cuda.synchronize()
+    rc.rc_stream_status()
+    assert_bits(to_host(flat[0], "f32"), host[0], "bucketer p=1")
+    b.close()

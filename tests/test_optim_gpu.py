@@ -206,3 +206,8 @@ def test_sharded_owner_broadcast_variant(rc):
         assert_bits(to_host(vv, "f32"), w_s[t], f"owner exp_avg_sq t={t}")
         for q in range(p):
             assert_bits(to_host(out[q], "f32"), want[t][q], f"owner broadcast t={t} rank {q}")
+
+
+def test_zero1_single_rank(rc):
+    """p = 1: no reduction partner; the step is AdamW on the whole vector (x scale)."""
+    _zero1_case(rc, 1, 4096 + 4, "f32", "bf16", seed=99)

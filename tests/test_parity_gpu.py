@@ -202,7 +202,8 @@ def test_ring_in_place(rc):
 
 # ------------------------------------------------------------ hierarchical
 @pytest.mark.parametrize("p,G,n", [(8, 4, 8 * 1024), (8, 2, 1000), (4, 2, 65536), (16, 4, 4096),
-                                   (6, 3, 999), (8, 1, 512), (8, 8, 512), (2, 2, 10)])
+                                   (6, 3, 999), (8, 1, 512), (8, 8, 512), (2, 2, 10),
+                                   (16, 8, 16 * 2048), (16, 2, 16 * 1024 + 64)])
 @pytest.mark.parametrize("dt", DTS)
 def test_hier(rc, p, G, n, dt):
     xs = _data(p, n, dt, seed=4000 + p * G + n)
