@@ -25,6 +25,8 @@ __all__ = [
     "rc_all_reduce", "rc_reduce_scatter", "rc_all_gather", "rc_reduce", "rc_broadcast",
     "rc_ring_all_reduce", "rc_ring_all_reduce_noalloc", "rc_hier_all_reduce", "rc_copy", "rc_reserve_workspace", "rc_check_buffer",
     "rc_probe_bounded_wait",
+    "rc_rank_all_reduce", "rc_rank_reduce_scatter", "rc_rank_all_gather", "rc_rank_ring_step",
+    "rc_ipc_handle", "rc_ipc_export", "rc_ipc_import", "rc_ipc_release",
     "rc_stream_status", "rc_launch_count", "rc_finalize", "rc_version", "rc_last_error",
 ]
 
@@ -87,6 +89,22 @@ _decl("rc_bucketer_ready", [_vp, _i, _vp])
 _decl("rc_bucketer_flush", [_vp, _vp])
 _decl("rc_bucketer_destroy", [_vp])
 _decl("rc_all_to_all_v", [_vpp, _vpp, _i, ctypes.POINTER(ctypes.c_size_t), _i, _vp])
+_decl("rc_rank_all_reduce", [_vpp, _vpp, _i, _i, _sz, _i, _i, _f, _vp])
+_decl("rc_rank_reduce_scatter", [_vpp, _vp, _i, _i, _sz, _i, _i, _i, _f, _vp])
+_decl("rc_rank_all_gather", [_vpp, _vp, _i, _i, _sz, _i, _vp])
+_decl("rc_rank_ring_step", [_vpp, _vpp, _vpp, _i, _i, _i, _sz, _i, _i, _f, _vp])
+
+
+class rc_ipc_handle(ctypes.Structure):
+    """Mirror of the C struct rc_ipc_handle (plain bytes: bytes(h) travels
+    between processes, rc_ipc_handle.from_buffer_copy(b) restores it)."""
+    _fields_ = [("ipc", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64), ("bytes", ctypes.c_uint64),
+                ("device", ctypes.c_int32), ("pid", ctypes.c_int32)]
+
+
+_decl("rc_ipc_export", [_vp, _sz, ctypes.POINTER(rc_ipc_handle)])
+_decl("rc_ipc_import", [ctypes.POINTER(rc_ipc_handle), ctypes.POINTER(_vp)])
+_decl("rc_ipc_release", [_vp])
 _decl("rc_reserve_workspace", [_sz, _vp])
 _decl("rc_check_buffer", [_vp, _sz])
 _decl("rc_probe_bounded_wait", [ctypes.c_uint64, _vp])
@@ -236,6 +254,73 @@ def rc_hier_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], group_size: int
     _check(lib.rc_hier_all_reduce(_ptrs(send), _ptrs(recv), p, group_size, _numel(send[0], n),
                                   _dt(dtype, send[0]), _op(op), scale, int(v), _stream(stream)),
            "rc_hier_all_reduce")
+
+
+# ---------------------------------------------------------------- rank view
+# One rank's share of a collective (rank-per-GPU execution): the buffer lists
+# hold the p ranks' buffers as this process addresses them -- its own tensor
+# and the other ranks' imported addresses (integers).  dtype and n are
+# required when the own buffer is a raw address.
+def _own(xs: Sequence, rank: int):
+    """The buffer that supplies n and dtype defaults: this rank's own (a
+    tensor), or the first one when rank is out of range (the library then
+    rejects the call)."""
+    return xs[rank] if 0 <= rank < len(xs) else xs[0]
+
+
+def rc_rank_all_reduce(send: Sequence[Buf], recv: Sequence[Buf], rank: int, n=None, dtype=None, op="sum",
+                       scale=1.0, stream=None):
+    p = len(send)
+    own = _own(send, rank)
+    _check(lib.rc_rank_all_reduce(_ptrs(send), _ptrs(recv), p, rank, _numel(own, n), _dt(dtype, own), _op(op),
+                                  scale, _stream(stream)), "rc_rank_all_reduce")
+
+
+def rc_rank_reduce_scatter(send: Sequence[Buf], recv_own: Buf, rank: int, n=None, in_dtype=None,
+                           out_dtype=None, op="sum", scale=1.0, stream=None):
+    p = len(send)
+    own = _own(send, rank)
+    _check(lib.rc_rank_reduce_scatter(_ptrs(send), _addr(recv_own), p, rank, _numel(own, n),
+                                      _dt(in_dtype, own), _dt(out_dtype, recv_own), _op(op), scale,
+                                      _stream(stream)), "rc_rank_reduce_scatter")
+
+
+def rc_rank_all_gather(send: Sequence[Buf], recv_own: Buf, rank: int, n=None, dtype=None, stream=None):
+    p = len(send)
+    _check(lib.rc_rank_all_gather(_ptrs(send), _addr(recv_own), p, rank, _numel(recv_own, n),
+                                  _dt(dtype, recv_own), _stream(stream)), "rc_rank_all_gather")
+
+
+def rc_rank_ring_step(send: Sequence[Buf], recv: Sequence[Buf], rank: int, step: int, ws=None, n=None,
+                      dtype=None, op="sum", scale=1.0, stream=None):
+    p = len(send)
+    own = _own(send, rank)
+    wsp = _ptrs(ws) if ws is not None else None
+    _check(lib.rc_rank_ring_step(_ptrs(send), _ptrs(recv), wsp, p, rank, step, _numel(own, n), _dt(dtype, own),
+                                 _op(op), scale, _stream(stream)), "rc_rank_ring_step")
+
+
+def rc_ipc_export(buf: Buf, nbytes=None) -> bytes:
+    """Describe a device buffer (tensor or address + nbytes) for another process."""
+    if nbytes is None:
+        if not _is_tensor(buf):
+            raise ValueError("nbytes is required for a raw address")
+        nbytes = buf.numel() * buf.element_size()
+    h = rc_ipc_handle()
+    _check(lib.rc_ipc_export(_addr(buf), int(nbytes), ctypes.byref(h)), "rc_ipc_export")
+    return bytes(h)
+
+
+def rc_ipc_import(handle: bytes) -> int:
+    """Map another process's exported buffer; returns its address here."""
+    h = rc_ipc_handle.from_buffer_copy(handle)
+    out = ctypes.c_void_p()
+    _check(lib.rc_ipc_import(ctypes.byref(h), ctypes.byref(out)), "rc_ipc_import")
+    return int(out.value)
+
+
+def rc_ipc_release(addr: int) -> None:
+    _check(lib.rc_ipc_release(int(addr)), "rc_ipc_release")
 
 
 def _hparams(lr, beta1, beta2, eps, weight_decay, step):

@@ -18,6 +18,8 @@
 #include <mutex>
 #include <vector>
 
+#include <unistd.h>
+
 #include "../../include/rankcoll.h"
 #include "common.cuh"
 #include "internal.h"
@@ -91,7 +93,9 @@ MemGetAddressRangeFn address_range_fn() {
 
 // [ptr, ptr+bytes) must be device (or managed) memory of the current device,
 // inside one allocation.
-rc_status check_device_range(const void *ptr, size_t bytes, const char *what, int idx) {
+// peer_ok: the memory may also belong to another device that the current
+// device can access (a peer mapping).
+rc_status check_device_range(const void *ptr, size_t bytes, const char *what, int idx, bool peer_ok = false) {
   if (ptr == nullptr) return fail(RC_ERR_INVALID_ARG, "%s[%d] is NULL", what, idx);
   cudaPointerAttributes at{};
   cudaError_t e = cudaPointerGetAttributes(&at, ptr);
@@ -104,9 +108,14 @@ rc_status check_device_range(const void *ptr, size_t bytes, const char *what, in
     return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p is not device memory", what, idx, ptr);
   int dev = -1;
   cudaGetDevice(&dev);
-  if (at.type == cudaMemoryTypeDevice && at.device != dev)
-    return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p lives on device %d, current device is %d", what, idx,
-                ptr, at.device, dev);
+  if (at.type == cudaMemoryTypeDevice && at.device != dev) {
+    int can = 0;
+    if (!peer_ok || cudaDeviceCanAccessPeer(&can, dev, at.device) != cudaSuccess || !can) {
+      cudaGetLastError();
+      return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p lives on device %d, current device is %d%s", what, idx,
+                  ptr, at.device, dev, peer_ok ? ", which cannot access it" : "");
+    }
+  }
   if (env_int("RC_SKIP_RANGE_CHECK", 0)) return RC_OK;
   MemGetAddressRangeFn fn = address_range_fn();
   if (fn) {
@@ -167,12 +176,12 @@ rc_status check_aliasing(const std::vector<Buf> &bs) {
   return RC_OK;
 }
 
-rc_status check_ranges(const std::vector<Buf> &bs) {
+rc_status check_ranges(const std::vector<Buf> &bs, bool peer_ok = false) {
   for (const Buf &b : bs) {
     if (b.esz > 1 && b.lo % (uintptr_t)b.esz != 0)
       return fail(RC_ERR_INVALID_ARG, "%s[%d]=%p is not aligned to its %d-byte elements", b.what, b.idx,
                   (void *)b.lo, b.esz);
-    rc_status st = check_device_range((const void *)b.lo, b.hi - b.lo, b.what, b.idx);
+    rc_status st = check_device_range((const void *)b.lo, b.hi - b.lo, b.what, b.idx, peer_ok);
     if (st != RC_OK) return st;
   }
   return RC_OK;
@@ -663,6 +672,242 @@ rc_status rc_all_to_all(const void *const *send, void *const *recv, int p, size_
   if (n % (size_t)p != 0) return fail(RC_ERR_INVALID_ARG, "n=%zu is not a multiple of p=%d", n, p);
   std::vector<size_t> counts((size_t)p * p, n / p);
   return rc_all_to_all_v(send, recv, p, counts.data(), dt, stream);
+}
+
+// ---------------------------------------------------------------- rank view
+rc_status rc_rank_all_reduce(const void *const *send, void *const *recv, int p, int rank, size_t n,
+                             rc_dtype dt, rc_op op, float scale, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(dt, dt, op, scale)) != RC_OK) return st;
+  if (rank < 0 || rank >= p) return fail(RC_ERR_INVALID_ARG, "rank=%d outside [0, %d)", rank, p);
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, s, 0, r, false, "send", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if ((st = check_ranges(bs, true)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  ReduceJob j{};
+  j.p = p;
+  j.n = n;
+  for (int r = 0; r < p; ++r) {
+    j.src[r] = send[r];
+    j.dst[r] = recv[r];
+  }
+  j.in_dt = j.out_dt = dt;
+  j.op = op;
+  j.scale = scale;
+  j.mode = kModeAll;
+  j.ndst = p;
+  j.c0 = rank;
+  j.c1 = rank + 1;
+  return launched(launch_reduce(j, (cudaStream_t)stream), "rank all_reduce launch");
+}
+
+rc_status rc_rank_reduce_scatter(const void *const *send, void *recv_own, int p, int rank, size_t n,
+                                 rc_dtype in_dt, rc_dtype out_dt, rc_op op, float scale,
+                                 rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(in_dt, out_dt, op, scale)) != RC_OK) return st;
+  if (rank < 0 || rank >= p) return fail(RC_ERR_INVALID_ARG, "rank=%d outside [0, %d)", rank, p);
+  if (n % (size_t)p != 0) return fail(RC_ERR_INVALID_ARG, "n=%zu is not a multiple of p=%d", n, p);
+  if (n == 0) return RC_OK;
+  if (!send) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const uint64_t m = n / p;
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, dt_size(in_dt), 0, r, false, "send", r));
+  bs.push_back(make_buf(recv_own, m, dt_size(out_dt), (uint64_t)rank * m, rank, true, "recv_own", 0));
+  if ((st = check_ranges(bs, true)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  ReduceJob j{};
+  j.p = p;
+  j.n = n;
+  // only chunk `rank` is computed, so only dst[rank] is ever written
+  for (int r = 0; r < p; ++r) {
+    j.src[r] = send[r];
+    j.dst[r] = recv_own;
+  }
+  j.in_dt = in_dt;
+  j.out_dt = out_dt;
+  j.op = op;
+  j.scale = scale;
+  j.mode = kModeScatter;
+  j.c0 = rank;
+  j.c1 = rank + 1;
+  return launched(launch_reduce(j, (cudaStream_t)stream), "rank reduce_scatter launch");
+}
+
+rc_status rc_rank_all_gather(const void *const *send, void *recv_own, int p, int rank, size_t n,
+                             rc_dtype dt, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if (!dt_ok(dt)) return fail(RC_ERR_INVALID_ARG, "unknown dtype");
+  if (rank < 0 || rank >= p) return fail(RC_ERR_INVALID_ARG, "rank=%d outside [0, %d)", rank, p);
+  if (n % (size_t)p != 0) return fail(RC_ERR_INVALID_ARG, "n=%zu is not a multiple of p=%d", n, p);
+  if (n == 0) return RC_OK;
+  if (!send) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  const int s = dt_size(dt);
+  const uint64_t m = n / p;
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], m, s, (uint64_t)r * m, r, false, "send", r));
+  bs.push_back(make_buf(recv_own, n, s, 0, rank, true, "recv_own", 0));
+  if ((st = check_ranges(bs, true)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  FanoutJob f{};
+  f.nsrc = p;
+  f.p = 1;  // one destination: this rank's output
+  f.src_bytes = m * s;
+  f.elem_bytes = s;
+  for (int r = 0; r < p; ++r) f.src[r] = send[r];
+  f.dst[0] = recv_own;
+  if ((const char *)recv_own + (uint64_t)rank * m * s == (const char *)send[rank]) f.skip[0] = 1u << rank;
+  return launched(launch_fanout(f, (cudaStream_t)stream), "rank all_gather launch");
+}
+
+rc_status rc_rank_ring_step(const void *const *send, void *const *recv, void *const *ws, int p, int rank,
+                            int step, size_t n, rc_dtype dt, rc_op op, float scale, rc_stream_t stream) {
+  rc_status st;
+  if ((st = check_p_n(p, n)) != RC_OK) return st;
+  if ((st = check_reduce_types(dt, dt, op, scale)) != RC_OK) return st;
+  if (p < 2) return fail(RC_ERR_INVALID_ARG, "the ring needs p >= 2 (p=%d)", p);
+  if (rank < 0 || rank >= p) return fail(RC_ERR_INVALID_ARG, "rank=%d outside [0, %d)", rank, p);
+  if (step < 0 || step >= 2 * (p - 1))
+    return fail(RC_ERR_INVALID_ARG, "step=%d outside [0, %d)", step, 2 * (p - 1));
+  if (n == 0) return RC_OK;
+  if (!send || !recv) return fail(RC_ERR_INVALID_ARG, "pointer array is NULL");
+  if (dt == RC_BF16 && !ws) return fail(RC_ERR_INVALID_ARG, "bf16 needs the ranks' workspaces (ws is NULL)");
+  const int s = dt_size(dt);
+  const uint64_t C = (n + p - 1) / p;
+  std::vector<Buf> bs;
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(send[r], n, s, 0, r, false, "send", r));
+  for (int r = 0; r < p; ++r) bs.push_back(make_buf(recv[r], n, s, 0, r, true, "recv", r));
+  if (dt == RC_BF16)
+    for (int r = 0; r < p; ++r) bs.push_back(make_buf(ws[r], 2 * C, 4, 0, r, true, "ws", r));
+  if ((st = check_ranges(bs, true)) != RC_OK) return st;
+  if ((st = check_aliasing(bs)) != RC_OK) return st;
+  RankStepJob j{};
+  j.p = p;
+  j.rank = rank;
+  j.step = step;
+  j.n = n;
+  j.dt = dt;
+  j.op = op;
+  j.scale = scale;
+  for (int r = 0; r < p; ++r) {
+    j.x[r] = send[r];
+    j.y[r] = recv[r];
+    j.ws[r] = dt == RC_BF16 ? ws[r] : nullptr;
+  }
+  return launched(launch_rank_ring_step(j, (cudaStream_t)stream), "rank ring step launch");
+}
+
+// ---------------------------------------------------------------- IPC
+namespace {
+struct IpcMap {
+  unsigned char key[sizeof(cudaIpcMemHandle_t)];
+  char *base;
+  size_t size;
+  int refs;
+};
+std::mutex g_ipc_mu;
+std::vector<IpcMap> g_ipc;
+static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(((rc_ipc_handle *)nullptr)->ipc),
+              "rc_ipc_handle.ipc must hold a cudaIpcMemHandle_t");
+}  // namespace
+
+rc_status rc_ipc_export(const void *ptr, size_t bytes, rc_ipc_handle *out) {
+  if (!out) return fail(RC_ERR_INVALID_ARG, "rc_ipc_export: out is NULL");
+  rc_status st = check_device_range(ptr, bytes, "ptr", 0);
+  if (st != RC_OK) return st;
+  MemGetAddressRangeFn fn = address_range_fn();
+  if (!fn) return fail(RC_ERR_UNSUPPORTED, "rc_ipc_export: allocation ranges cannot be queried");
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (fn(&base, &size, (CUdeviceptr)(uintptr_t)ptr) != CUDA_SUCCESS)
+    return fail(RC_ERR_INVALID_ARG, "rc_ipc_export: %p is not inside a device allocation", ptr);
+  cudaIpcMemHandle_t h;
+  cudaError_t e = cudaIpcGetMemHandle(&h, (void *)(uintptr_t)base);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "cudaIpcGetMemHandle");
+  }
+  int dev = -1;
+  cudaGetDevice(&dev);
+  memset(out, 0, sizeof *out);
+  memcpy(out->ipc, &h, sizeof h);
+  out->offset = (uint64_t)((uintptr_t)ptr - (uintptr_t)base);
+  out->bytes = bytes;
+  out->device = dev;
+  out->pid = (int32_t)getpid();
+  return RC_OK;
+}
+
+rc_status rc_ipc_import(const rc_ipc_handle *h, void **ptr) {
+  if (!h || !ptr) return fail(RC_ERR_INVALID_ARG, "rc_ipc_import: NULL argument");
+  *ptr = nullptr;
+  if (h->pid == (int32_t)getpid())
+    return fail(RC_ERR_INVALID_ARG, "rc_ipc_import: the handle was exported by this process; use the buffer itself");
+  std::lock_guard<std::mutex> lock(g_ipc_mu);
+  for (IpcMap &m : g_ipc) {
+    if (memcmp(m.key, h->ipc, sizeof m.key) == 0) {
+      if (h->offset > m.size || h->bytes > m.size - h->offset)
+        return fail(RC_ERR_INVALID_ARG, "rc_ipc_import: offset %llu + %llu bytes past the mapped allocation (%zu)",
+                    (unsigned long long)h->offset, (unsigned long long)h->bytes, m.size);
+      ++m.refs;
+      *ptr = m.base + h->offset;
+      return RC_OK;
+    }
+  }
+  cudaIpcMemHandle_t hh;
+  memcpy(&hh, h->ipc, sizeof hh);
+  void *base = nullptr;
+  cudaError_t e = cudaIpcOpenMemHandle(&base, hh, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "cudaIpcOpenMemHandle");
+  }
+  size_t size = (size_t)-1;
+  MemGetAddressRangeFn fn = address_range_fn();
+  CUdeviceptr b = 0;
+  if (fn && fn(&b, &size, (CUdeviceptr)(uintptr_t)base) != CUDA_SUCCESS) size = (size_t)-1;
+  if (h->offset > size || h->bytes > size - h->offset) {
+    cudaIpcCloseMemHandle(base);
+    return fail(RC_ERR_INVALID_ARG, "rc_ipc_import: offset %llu + %llu bytes past the mapped allocation (%zu)",
+                (unsigned long long)h->offset, (unsigned long long)h->bytes, size);
+  }
+  IpcMap m;
+  memcpy(m.key, h->ipc, sizeof m.key);
+  m.base = static_cast<char *>(base);
+  m.size = size;
+  m.refs = 1;
+  g_ipc.push_back(m);
+  *ptr = m.base + h->offset;
+  return RC_OK;
+}
+
+rc_status rc_ipc_release(void *ptr) {
+  std::lock_guard<std::mutex> lock(g_ipc_mu);
+  const char *q = static_cast<const char *>(ptr);
+  // the mapping that contains ptr; an address one past the end belongs to a
+  // mapping only if no mapping starts there (an empty buffer at the end)
+  size_t hit = g_ipc.size();
+  for (size_t i = 0; i < g_ipc.size() && hit == g_ipc.size(); ++i)
+    if (q >= g_ipc[i].base && (size_t)(q - g_ipc[i].base) < g_ipc[i].size) hit = i;
+  for (size_t i = 0; i < g_ipc.size() && hit == g_ipc.size(); ++i)
+    if (q >= g_ipc[i].base && (size_t)(q - g_ipc[i].base) == g_ipc[i].size) hit = i;
+  if (hit == g_ipc.size()) return fail(RC_ERR_INVALID_ARG, "rc_ipc_release: %p is not an imported buffer", ptr);
+  IpcMap &m = g_ipc[hit];
+  if (--m.refs > 0) return RC_OK;
+  cudaError_t e = cudaIpcCloseMemHandle(m.base);
+  g_ipc.erase(g_ipc.begin() + (long)hit);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "cudaIpcCloseMemHandle");
+  }
+  return RC_OK;
 }
 
 rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream) {

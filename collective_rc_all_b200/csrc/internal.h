@@ -28,6 +28,9 @@ struct ReduceJob {
   float scale;
   int mode;
   int ndst;  // kModeAll: number of outputs (0 means p)
+  // Chunks [c0, c1) only (chunk length ceil(n/p)); c1 = 0 means all p.  A
+  // rank's share of a collective is its own chunk.
+  int c0, c1;
 };
 
 // A p-source fold over aligned 16-byte vectors (fold.cu).  G = p is the flat
@@ -68,6 +71,18 @@ struct HierJob {
   void *y[kMaxP];
   void *ws;  // staged variant: (ng + 1) * n accumulator values
   int p, G;
+  uint64_t n;
+  int dt, op;
+  float scale;
+};
+
+// One step of the literal ring as executed by receiving rank `rank` (rank.cu):
+// the p ranks' buffers as this process addresses them (own or peer-mapped).
+struct RankStepJob {
+  const void *x[kMaxP];  // send
+  void *y[kMaxP];        // recv
+  void *ws[kMaxP];       // bf16: each rank's 2 * ceil(n/p) fp32 partials
+  int p, rank, step;
   uint64_t n;
   int dt, op;
   float scale;
@@ -115,6 +130,7 @@ cudaError_t noalloc_scratch_ptr(void **out);
 cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s);
 cudaError_t launch_hier_staged(const HierJob &job, cudaStream_t s);
 cudaError_t launch_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);
+cudaError_t launch_rank_ring_step(const RankStepJob &job, cudaStream_t s);
 cudaError_t launch_zero1(const Zero1Job &job, cudaStream_t s);
 cudaError_t launch_all_to_all(const A2aJob &job, cudaStream_t s);
 cudaError_t launch_adamw(float *param, float *exp_avg, float *exp_avg_sq, const void *grad, int grad_dt,

@@ -47,6 +47,7 @@ struct ReduceParams {
   int p;
   int mode;
   int ndst;  // outputs in kModeAll
+  int c0;    // first chunk of the launch (chunk range [c0, c1))
 };
 
 __device__ __forceinline__ int rot(uint64_t c, int k, int p) {
@@ -64,8 +65,10 @@ __global__ void __launch_bounds__(kNT) rc_reduce_scalar_kernel(const __grid_cons
   pdl_trigger();
   const int p = a.p;
   const uint64_t G = gridDim.x;
-  uint64_t u0 = a.nvec * blockIdx.x / G;
-  const uint64_t u1 = a.nvec * (blockIdx.x + 1) / G;
+  // a.nvec elements starting at element c0 * C (the launch's chunk range)
+  const uint64_t lo = (uint64_t)a.c0 * a.C;
+  uint64_t u0 = lo + a.nvec * blockIdx.x / G;
+  const uint64_t u1 = lo + a.nvec * (blockIdx.x + 1) / G;
   while (u0 < u1) {
     // all elements in [u0, useg) share chunk c, hence one fold order
     const uint64_t c = u0 / a.C;
@@ -103,8 +106,9 @@ __global__ void __launch_bounds__(kNT) rc_reduce_front_kernel(const __grid_const
   constexpr int VEC = kVec<TI>;
   const int p = a.p;
   const uint64_t cvec = a.C / VEC;
-  const uint64_t c = blockIdx.x / tiles_per_chunk;
-  const uint64_t v0 = c * cvec + (blockIdx.x - c * tiles_per_chunk) * (uint64_t)(kNT * ILP);
+  const uint64_t cl = blockIdx.x / tiles_per_chunk;  // chunk within the launch's range
+  const uint64_t c = a.c0 + cl;
+  const uint64_t v0 = c * cvec + (blockIdx.x - cl * tiles_per_chunk) * (uint64_t)(kNT * ILP);
   const uint64_t cend = (c + 1) * cvec;
   const uint64_t vend = cend < a.nvec ? cend : a.nvec;
   if (v0 >= vend) return;
@@ -156,12 +160,12 @@ __global__ void __launch_bounds__(kNT) rc_reduce_front_kernel(const __grid_const
 // chunk) -- one small CTA, scalar.
 template <int PMAX, class TI, class TO, int OP>
 __global__ void __launch_bounds__(32) rc_reduce_tail_kernel(const __grid_constant__ ReduceParams a,
-                                                          uint64_t first) {
+                                                          uint64_t first, uint64_t last) {
   using Acc = typename TI::Acc;
   pdl_wait();
   pdl_trigger();
   const int p = a.p;
-  for (uint64_t e = first + threadIdx.x; e < a.n; e += blockDim.x) {
+  for (uint64_t e = first + threadIdx.x; e < last; e += blockDim.x) {
     const uint64_t c = e / a.C;
     Acc acc = load_elem<TI>(a.src[rot(c, 0, p)], e);
     for (int k = 1; k < p; ++k) acc = combine<OP>(acc, load_elem<TI>(a.src[rot(c, k, p)], e));
@@ -186,6 +190,12 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
   a.mode = job.mode;
   a.scale = job.scale;
   a.ndst = job.mode == kModeAll ? (job.ndst > 0 ? job.ndst : p) : 1;
+  const int c0 = job.c0, c1 = job.c1 > 0 ? job.c1 : p;
+  if (c0 < 0 || c0 >= c1 || c1 > p) return cudaErrorInvalidValue;
+  a.c0 = c0;
+  const bool whole = (c0 == 0 && c1 == p);
+  const uint64_t e_lo = std::min<uint64_t>(n, (uint64_t)c0 * C);  // the range's elements
+  const uint64_t e_hi = std::min<uint64_t>(n, (uint64_t)c1 * C);
   bool aligned = true;
   for (int r = 0; r < p; ++r) {
     a.src[r] = static_cast<const char *>(job.src[r]);
@@ -221,25 +231,28 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
   // (RC_AR_FOLD=1): with one vector per thread the register front kernel
   // measured faster for the p = 8 x 8 MiB fp32 all-reduce (23.4 vs 25.3 us
   // back to back, 20.5 vs 23.6 us alone).
-  if (vector && job.mode == kModeAll && env_int("RC_AR_FOLD", 0) && fold_tma_eligible(f)) {
+  if (whole && vector && job.mode == kModeAll && env_int("RC_AR_FOLD", 0) && fold_tma_eligible(f)) {
     // the staged fold covers whole vectors; the tail (n % VEC elements) is scalar
     if ((err = launch_fold_tma(f, s)) != cudaSuccess) return err;
     a.nvec = n / VEC;
     if (a.nvec * VEC < n) {
       if ((err = launch_kernel(rc_reduce_tail_kernel<PMAX, TI, TO, OP>, dim3(1), dim3(32), 0, s, a,
-                               a.nvec * VEC)) != cudaSuccess)
+                               a.nvec * VEC, n)) != cudaSuccess)
         return err;
     }
     return cudaSuccess;
   }
+  if (e_lo == e_hi) return cudaSuccess;  // the range holds no element
   if (vector) {
     a.nvec = n / VEC;
-    if (a.nvec > 0) {
+    // whole vectors of the range: chunks are whole vectors, so only the last
+    // chunk of the vector can end in a partial one
+    if (std::min<uint64_t>(a.nvec * VEC, e_hi) > e_lo) {
       const uint64_t cvec = C / VEC;
       auto go = [&](auto ilp_tag) -> cudaError_t {
         constexpr int ILP = decltype(ilp_tag)::value;
         const uint64_t tpc = (cvec + kNT * ILP - 1) / (kNT * ILP);
-        const uint64_t grid = tpc * (uint64_t)p;
+        const uint64_t grid = tpc * (uint64_t)(c1 - c0);
         if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
         return launch_kernel(rc_reduce_front_kernel<PMAX, TI, TO, OP, ILP>, dim3((unsigned)grid), dim3(kNT), 0,
                              s, a, tpc);
@@ -251,9 +264,10 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
       err = ilp == 1 ? go(std::integral_constant<int, 1>()) : go(std::integral_constant<int, 2>());
       if (err != cudaSuccess) return err;
     }
-    if (a.nvec * VEC < n) {
-      if ((err = launch_kernel(rc_reduce_tail_kernel<PMAX, TI, TO, OP>, dim3(1), dim3(32), 0, s, a,
-                               a.nvec * VEC)) != cudaSuccess)
+    const uint64_t t0 = std::max<uint64_t>(a.nvec * VEC, e_lo);
+    if (t0 < e_hi) {
+      if ((err = launch_kernel(rc_reduce_tail_kernel<PMAX, TI, TO, OP>, dim3(1), dim3(32), 0, s, a, t0,
+                               e_hi)) != cudaSuccess)
         return err;
     }
   } else {
@@ -261,8 +275,8 @@ cudaError_t run(const ReduceJob &job, cudaStream_t s) {
     int occ = 0;
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNT, 0);
     if (err != cudaSuccess) return err;
-    a.nvec = n;
-    uint64_t grid = std::min<uint64_t>((uint64_t)sms * std::max(occ, 1), (n + kNT - 1) / kNT);
+    a.nvec = e_hi - e_lo;  // elements, from c0 * C
+    uint64_t grid = std::min<uint64_t>((uint64_t)sms * std::max(occ, 1), (a.nvec + kNT - 1) / kNT);
     grid = std::max<uint64_t>(grid, 1);
     if ((err = launch_kernel(kern, dim3((unsigned)grid), dim3(kNT), 0, s, a)) != cudaSuccess) return err;
   }

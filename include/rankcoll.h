@@ -43,6 +43,13 @@
  *         到专家输出" -- dispatch towards the experts and combine back, split
  *         counts tell the receiver how much arrives; section "为什么 top-k 和 EP
  *         degree 会直接放大通信" -- payload t*k*h*b per rank and phase.
+ *  [P2P]  "分布式训练/推理", section "从单卡到多卡：瓶颈从 HBM 扩展到互联" -- past
+ *         one GPU the ranks' data crosses NVLink/NVSwitch, a transfer costs
+ *         alpha + bytes/bandwidth; section "通信原语：rank、world size 和
+ *         collective operations" -- a rank is usually one GPU or one process;
+ *         section "PyTorch distributed：代码里真正发生了什么" -- the collective
+ *         library turns a collective into GPU kernels that move data between
+ *         GPUs; section "Ring all-reduce 的带宽账" -- T_AR = 2(N-1)/N * S/W.
  *  [HIER] "大模型并行的最小闭环：集合通信、TP、FSDP/ZeRO-3 到权重分片", log excerpt
  *         "分层 AllReduce + SHARP", steps 1-6 -- intra-node AllReduce, one
  *         representative per node, the node results added together, intra-node
@@ -334,6 +341,101 @@ rc_status rc_zero1_step(const void *const *grads, void *const *params, float *co
                         float *const *exp_avg, float *const *exp_avg_sq, int p, size_t n,
                         rc_dtype grad_dt, rc_dtype param_dt, float scale,
                         const rc_adamw_hparams *hp, rc_stream_t stream);
+
+/*
+ * Rank view [P2P]: one rank's share of a collective, for rank-per-GPU
+ * execution -- one process per GPU, each reaching the other ranks' buffers
+ * through peer mappings (rc_ipc_import).  The pointer arrays hold the p
+ * ranks' buffers as the calling process addresses them: its own buffer at
+ * index `rank`, the other ranks' mapped buffers elsewhere.  A pointer may
+ * live on another device when the current device can access that device's
+ * memory (an imported mapping always can).
+ *
+ * Calling a rank-view function once for every rank 0..p-1 gives exactly the
+ * bits of the corresponding whole collective above (same chunks, same fold
+ * order).  The functions do not synchronise the ranks: the caller must make
+ * every rank's inputs complete before any rank's call runs, and every rank's
+ * call complete before the outputs are read or the inputs reused (for
+ * example: synchronise the stream, then a host barrier among the processes).
+ * Validation is as for the whole collective.
+ */
+
+/* Chunk `rank` of the all-reduce (elements [rank*C, min((rank+1)*C, n)),
+ * C = ceil(n/p)): read from the p send buffers, folded in the ring order,
+ * scaled, written to the same elements of all p recv buffers.  Traffic per
+ * rank: (p-1)/p * n elements read from peers and as many written to them.
+ * (The pull form of the one-shot all-reduce, where a rank reads the whole
+ * vector from every peer and writes only its own output, is
+ * rc_reduce(send, recv_own, p, root = rank, ...).) */
+rc_status rc_rank_all_reduce(const void *const *send, void *const *recv, int p, int rank, size_t n,
+                             rc_dtype dt, rc_op op, float scale, rc_stream_t stream);
+
+/* recv_own (n/p elements of out_dt) = shard `rank` of the reduce-scatter,
+ * read from chunk `rank` of the p send buffers (n elements each, n % p == 0).
+ * recv_own may be send[rank] + rank*(n/p) with equal element sizes. */
+rc_status rc_rank_reduce_scatter(const void *const *send, void *recv_own, int p, int rank, size_t n,
+                                 rc_dtype in_dt, rc_dtype out_dt, rc_op op, float scale,
+                                 rc_stream_t stream);
+
+/* recv_own (n elements) = the concatenation of the p shards send[0..p-1]
+ * (n/p elements each): every rank pulls the others' shards.  If
+ * recv_own + rank*(n/p) == send[rank] the own shard is left in place. */
+rc_status rc_rank_all_gather(const void *const *send, void *recv_own, int p, int rank, size_t n,
+                             rc_dtype dt, rc_stream_t stream);
+
+/* Step `step` in [0, 2(p-1)) of the literal ring all-reduce [RING], as
+ * executed by receiving rank `rank` (p >= 2), which pulls from its
+ * predecessor r = rank-1 mod p:
+ *  - reduce-scatter step k = step < p-1, chunk c = (rank-k-2) mod p:
+ *    partial_rank[c] = msg (+) send[rank][chunk c], where msg is
+ *    send[r][chunk c] at k = 0 and r's partial of chunk c after; at
+ *    k = p-2 (c == rank) recv[rank][chunk rank] = cast(scale * acc) instead.
+ *  - all-gather step k = step - (p-1), chunk c = (rank-k-1) mod p:
+ *    recv[rank][chunk c] = recv[r][chunk c].
+ * Partials are fp32 (int32 for int32).  For fp32 and int32 they live in the
+ * receiver's recv buffer (chunk c); for bf16 in ws[rank], 2*C floats per
+ * rank (C = ceil(n/p)), slot step%2.  ws may be NULL unless dt is bf16.
+ * Step s of every rank must be complete before any rank starts step s+1;
+ * all steps of all ranks give exactly rc_ring_all_reduce(..., LITERAL). */
+rc_status rc_rank_ring_step(const void *const *send, void *const *recv, void *const *ws, int p, int rank,
+                            int step, size_t n, rc_dtype dt, rc_op op, float scale, rc_stream_t stream);
+
+/*
+ * Peer mappings between processes (CUDA IPC) [P2P].  rc_ipc_export describes
+ * a device buffer so that another process can map it; rc_ipc_import maps
+ * such a description into the calling process (enabling peer access from the
+ * current device when the buffer lives on another one) and returns the
+ * buffer's address there; rc_ipc_release unmaps it.  The handle is plain
+ * bytes and may travel through any channel (a torch.distributed object
+ * gather, a file, a socket).
+ *
+ * A buffer inside a larger allocation (a caching allocator's block) is
+ * exported as that allocation plus an offset; importing maps the whole
+ * allocation once per process (several imports of buffers in one allocation
+ * share the mapping, reference-counted) and returns base + offset.  The
+ * exporting process must keep the allocation alive until every importer has
+ * released it.  A process cannot import its own export (RC_ERR_INVALID_ARG):
+ * use the buffer's own address.
+ */
+typedef struct {
+  unsigned char ipc[64];  /* the driver's IPC handle of the containing allocation */
+  uint64_t offset;        /* buffer address - allocation base */
+  uint64_t bytes;         /* buffer length */
+  int32_t device;         /* exporting device ordinal (in the exporter's numbering) */
+  int32_t pid;            /* exporting process */
+} rc_ipc_handle;
+
+/* [ptr, ptr+bytes) must be device memory of the current device inside one
+ * allocation (rc_check_buffer). */
+rc_status rc_ipc_export(const void *ptr, size_t bytes, rc_ipc_handle *out);
+
+/* *ptr = the exported buffer's address in this process. */
+rc_status rc_ipc_import(const rc_ipc_handle *h, void **ptr);
+
+/* Drop one import of the buffer at ptr (an address rc_ipc_import returned);
+ * the allocation's mapping is closed with its last import.  Synchronises
+ * nothing: the caller makes sure no work on the mapping is pending. */
+rc_status rc_ipc_release(void *ptr);
 
 /*
  * Plain device copy dst[0, bytes) = src[0, bytes) with this library's

@@ -113,3 +113,25 @@ def test_optimizer_arguments_rejected_on_host(rc):
     assert L.rc_zero1_step(a, a, a, a, a, 8, 0, 0, 1, 0.125, ctypes.byref(hp), None) == 0   # empty
     assert L.rc_adamw_step(None, None, None, None, 0, 0, ctypes.byref(hp), None) == 0
     assert rc.rc_launch_count() == before
+
+
+def test_rank_view_and_ipc_arguments_rejected_on_host(rc):
+    L = rc.lib
+    a = _null(8)
+    before = rc.rc_launch_count()
+    assert L.rc_rank_all_reduce(a, a, 4, 4, 10, 0, 0, 1.0, None) == 1          # rank == p
+    assert L.rc_rank_all_reduce(a, a, 4, -1, 10, 0, 0, 1.0, None) == 1         # rank < 0
+    assert L.rc_rank_all_reduce(a, a, 4, 0, 10, 0, 1, 0.5, None) == 1          # scale with MAX
+    assert L.rc_rank_all_reduce(a, a, 4, 0, 10, 0, 0, 1.0, None) == 1          # NULL buffers
+    assert L.rc_rank_reduce_scatter(a, None, 4, 0, 10, 0, 0, 0, 1.0, None) == 1  # 4 does not divide 10
+    assert L.rc_rank_all_gather(a, None, 4, 5, 8, 0, None) == 1                # rank out of range
+    assert L.rc_rank_ring_step(a, a, None, 1, 0, 0, 10, 0, 0, 1.0, None) == 1  # the ring needs p >= 2
+    assert L.rc_rank_ring_step(a, a, None, 4, 0, 6, 10, 0, 0, 1.0, None) == 1  # step 6 of 2(p-1) = 6
+    assert L.rc_rank_ring_step(a, a, None, 4, 0, 0, 10, 1, 0, 1.0, None) == 1  # bf16 without workspaces
+    assert "workspace" in rc.rc_last_error()
+    assert L.rc_rank_all_reduce(a, a, 4, 0, 0, 0, 0, 1.0, None) == 0           # n = 0: nothing to do
+    assert L.rc_ipc_import(None, None) == 1
+    assert L.rc_ipc_release(None) == 1                                          # never imported
+    h = rc.rc_ipc_handle()
+    assert L.rc_ipc_export(None, 16, ctypes.byref(h)) == 1                      # NULL buffer
+    assert rc.rc_launch_count() == before
