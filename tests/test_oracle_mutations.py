@@ -33,6 +33,11 @@ MUTANTS = {
     "bf16_ties_round_up": [("if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u) != 0u))", "if (lo >= 0x8000u)")],
     "ring_receiver_operands_swapped": [("combine(msg[r][i - b], w[d][i], is_int, op)", "combine(w[d][i], msg[r][i - b], is_int, op)")],
     "ring_allgather_wrong_chunk": [("size_t c = (size_t)(((r - k) % p + p) % p);", "size_t c = (size_t)(((r - k - 1) % p + p) % p);")],
+    "hier_leader_sum_starts_at_own_group": [("int g = (int)((c + 1) % (size_t)ng);", "int g = (int)(c % (size_t)ng);"),
+                                            ("g = (int)((c + 1 + (size_t)k) % (size_t)ng);",
+                                             "g = (int)((c + (size_t)k) % (size_t)ng);")],
+    "ring_reduce_scatter_chunk_shifted": [("size_t c = (size_t)(((r - k - 1) % q + q) % q);",
+                                           "size_t c = (size_t)(((r - k) % q + q) % q);")],
     "hier_group_drops_a_rank": [("ring_core(send + (size_t)g * (size_t)G, G,", "ring_core(send + (size_t)g * (size_t)G, G > 1 ? G - 1 : G,")],
     "adamw_no_first_bias_correction": [("float mhat = mi / bc1;", "float mhat = mi;")],
     "adamw_eps_inside_sqrt": [("float den = sqrtf(vhat) + eps;", "float den = sqrtf(vhat + eps);")],

@@ -272,6 +272,29 @@ def test_hier_vs_flat(oracle_mod, p, G):
                 assert np.all(np.abs(hf - ff) <= p * 2.0 ** -24 * xa + ulp)
 
 
+@pytest.mark.parametrize("G", [2, 3])
+def test_hier_order_closed_form(oracle_mod, G):
+    """Hand-derived values where only the two-level ring order gives the
+    right bits (p = 6).  Element 0 lies in chunk 0 at both levels, so a
+    group of size G folds its local ranks 1, 2, ..., 0 and the leaders fold
+    groups 1, 2, ..., 0.  With a = 2^24: (a + 1) rounds to a (tie to even),
+    so (a + 1) + (-a) = 0, while any other association of {a, 1, -a} gives 1.
+    G = 2 (three groups) puts a, 1, -a in groups 1, 2, 0; G = 3 (one group
+    of three ranks with the result) puts them on local ranks 1, 2, 0."""
+    p, n, a = 6, 6, np.float32(2.0 ** 24)
+    xs = [np.zeros(n, np.float32) for _ in range(p)]
+    if G == 2:   # group g = ranks 2g, 2g+1; S_g = x_{2g+1} + x_{2g}
+        xs[3][0], xs[5][0], xs[1][0] = a, 1.0, -a
+    else:        # group 0 = ranks 0, 1, 2 folded 1, 2, 0; group 1 is zero
+        xs[1][0], xs[2][0], xs[0][0] = a, 1.0, -a
+    for y in oracle_mod.hier_all_reduce(xs, G):
+        assert y[0] == 0.0 and not np.signbit(y[0])
+    # the flat ring order (ranks 1, 2, 3, 4, 5, 0) over the same data: for
+    # G = 2 it meets -a first and ends at 1; for G = 3 it matches the groups'
+    flat = oracle_mod.all_reduce(xs)[0][0]
+    assert flat == (1.0 if G == 2 else 0.0)
+
+
 def test_hier_degenerate_groups_equal_flat(oracle_mod):
     """G = p (one group) and G = 1 (p groups of one) are the flat ring order."""
     p, n = 8, 4096
