@@ -53,6 +53,11 @@ MUTANTS = {
                                     "for (int k = 0; k <= q && k < p - 1; ++k)\n                soff += counts[(size_t)r * p + k];")],
     "a2a_transposed_count": [("uint64_t c = counts[(size_t)r * p + q];", "uint64_t c = counts[(size_t)q * p + r];")],
     "a2a_traffic_swapped": [("traffic[r == q ? 0 : 1] += c * (uint64_t)esz;", "traffic[r == q ? 1 : 0] += c * (uint64_t)esz;")],
+    "reduce_at_chunk_from_index_count": [("acc_t a = fold_ring_order(send, p, n, (size_t)idx[j], in_dt, op);",
+                                          "acc_t a = fold_ring_order(send, p, k, (size_t)idx[j], in_dt, op);")],
+    "reduce_at_scale_dropped": [("store_result(out, j, out_dt, a, scale);", "store_result(out, j, out_dt, a, 1.0f);")],
+    "reduce_at_accepts_index_n": [("if (idx[j] >= n)\n            return RCO_EINVAL;",
+                                   "if (idx[j] > n)\n            return RCO_EINVAL;")],
     "int_sum_saturates": [("acc.i = (int32_t)((uint32_t)acc.i + (uint32_t)v.i);",
                            "{ long long t = (long long)acc.i + v.i; acc.i = t > 2147483647LL ? 2147483647 : (t < -2147483648LL ? (int32_t)-2147483648LL : (int32_t)t); }")],
 }

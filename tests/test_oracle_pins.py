@@ -356,3 +356,101 @@ def test_invalid_arguments(oracle_mod):
         oracle_mod.reduce(xs, root=4)
     with pytest.raises(oracle_mod.OracleError):
         oracle_mod.hier_all_reduce(xs, 3)
+
+
+# ---------------------------------------------------------------- sampled form
+# reduce_at(xs, idx) returns y[idx[j]] for selected indices only; the GPU tests
+# use it as the checker for full-size outputs.  Its own loop, index check and
+# output store are pinned here: by the hand-derived ring-order case, by the
+# closed forms, and by agreement with the pinned all_reduce / reduce_scatter
+# (y = sum_r x_r of "分布式训练/推理", section "通信原语：rank、world size 和
+# collective operations", in the ring order of "LLM Parallelism 基础", section
+# "Ring AllReduce").
+def _boundaries(n, p):
+    """Every chunk boundary +-1, the first and the last index, clipped to [0, n)."""
+    C = -(-n // p)
+    idx = {0, n - 1}
+    for c in range(1, p + 1):
+        for d in (-1, 0, 1):
+            if 0 <= c * C + d < n:
+                idx.add(c * C + d)
+    return np.array(sorted(idx), np.uint64)
+
+
+def test_reduce_at_ring_order_golden(oracle_mod):
+    """The hand-derived ring-order case, sampled in a shuffled order with a
+    repeated index: every element is 0 in ring order (2 in rank order)."""
+    g = golden("ring_order_fp32.json")
+    xs = [np.array(v, np.float32) for v in g["inputs"]]
+    idx = np.array([3, 0, 2, 1, 0], np.uint64)
+    got = oracle_mod.reduce_at(xs, idx)
+    assert got.tolist() == [g["all_reduce_sum"][int(i)] for i in idx]
+    assert got.dtype == np.float32
+
+
+@pytest.mark.parametrize("p", [1, 2, 3, 5, 8, 16])
+@pytest.mark.parametrize("n", [1, 7, 1000, 4099])
+def test_reduce_at_closed_form(oracle_mod, p, n):
+    """x_r[i] = i + r: y[i] = p*i + p(p-1)/2, max i + p - 1, min i, at every
+    chunk boundary +-1 and at random indices, in the order asked for."""
+    i = np.arange(n)
+    rng = np.random.default_rng(p * 7919 + n)
+    idx = np.concatenate([_boundaries(n, p), rng.integers(0, n, 64, dtype=np.uint64)])
+    rng.shuffle(idx)
+    ii = idx.astype(np.int64)
+    xs = [(i + r).astype(np.float32) for r in range(p)]
+    want = (p * ii + p * (p - 1) // 2).astype(np.float32)
+    assert_bits_equal(oracle_mod.reduce_at(xs, idx), want)
+    assert_bits_equal(oracle_mod.reduce_at(xs, idx, op="max"), (ii + p - 1).astype(np.float32))
+    assert_bits_equal(oracle_mod.reduce_at(xs, idx, op="min"), ii.astype(np.float32))
+    xi = [(i + r).astype(np.int32) for r in range(p)]
+    assert_bits_equal(oracle_mod.reduce_at(xi, idx, "i32"), want.astype(np.int32))
+    if p & (p - 1) == 0:
+        # AVG as x 1/p (exact for a power of two), narrowed once to bf16:
+        # torch's fp32 -> bf16 cast is round-to-nearest-even
+        avg = ((p * ii + p * (p - 1) // 2) / p).astype(np.float32)
+        ref = torch.from_numpy(avg).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        got = oracle_mod.reduce_at(xs, idx, "f32", "bf16", scale=1.0 / p)
+        assert got.dtype == np.uint16
+        assert_bits_equal(got, ref)
+
+
+@pytest.mark.parametrize("dt", DTS)
+@pytest.mark.parametrize("p,n", [(2, 63), (3, 100), (4, 1000), (7, 4097), (8, 4096), (16, 1023)])
+def test_reduce_at_matches_all_reduce(oracle_mod, dt, p, n):
+    """Order-sensitive random data: the sampled values equal the all-reduce's
+    at every chunk boundary +-1 and at shuffled random indices, every op."""
+    xs = _data(p, n, dt, seed=31 * p + n)
+    rng = np.random.default_rng(n)
+    idx = np.concatenate([_boundaries(n, p), rng.integers(0, n, 200, dtype=np.uint64)])
+    rng.shuffle(idx)
+    for op in OPS:
+        full = oracle_mod.all_reduce(xs, dt, op)[0]
+        assert_bits_equal(oracle_mod.reduce_at(xs, idx, dt, op=op), full[idx.astype(np.int64)])
+
+
+@pytest.mark.parametrize("p,n", [(2, 64), (4, 4096), (8, 8192), (16, 2048)])
+def test_reduce_at_matches_reduce_scatter_cast(oracle_mod, p, n):
+    """fp32 gradients -> bf16 with scale 1/p (the fused reduce_scatter of the
+    FSDP step): the sampled values equal the reduce_scatter's shards."""
+    xs = rc_inputs.normal(p, n, seed=40 + p, sigma=1e-3)
+    rs = np.concatenate(oracle_mod.reduce_scatter(xs, "f32", "bf16", "sum", 1.0 / p))
+    idx = np.concatenate([_boundaries(n, p), np.arange(0, n, 3, dtype=np.uint64)])
+    got = oracle_mod.reduce_at(xs, idx, "f32", "bf16", "sum", 1.0 / p)
+    assert_bits_equal(got, rs[idx.astype(np.int64)])
+    # and every index at once, in order
+    assert_bits_equal(oracle_mod.reduce_at(xs, np.arange(n, dtype=np.uint64), "f32", "bf16", "sum",
+                                           1.0 / p), rs)
+
+
+def test_reduce_at_index_range(oracle_mod):
+    """Index n is past the end and is rejected; n - 1 and no index at all are fine."""
+    p, n = 4, 10
+    xs = rc_inputs.uniform(p, n, seed=0)
+    full = oracle_mod.all_reduce(xs)[0]
+    assert_bits_equal(oracle_mod.reduce_at(xs, np.array([n - 1], np.uint64)), full[-1:])
+    assert oracle_mod.reduce_at(xs, np.zeros(0, np.uint64)).size == 0
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.reduce_at(xs, np.array([0, n], np.uint64))
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.reduce_at(xs, np.array([1], np.uint64), op="max", scale=0.5)
