@@ -54,6 +54,9 @@ UNIT = "GB/s"
 P, N = 8, 2097152
 SEED = 1
 SIGMA = 1e-2
+# B200 HBM bandwidth as the pages quote it ("分布式训练/推理", section "从单卡到多卡：
+# 瓶颈从 HBM 扩展到互联"): context beside the measured copy peak, not the roofline.
+PAGES_HBM_GBS = 8000.0
 FLUSH_BYTES = 512 << 20      # written, then...
 CLEAN_BYTES = 256 << 20      # ...a separate buffer read, so L2 is left holding clean lines
 WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 fp32 "
@@ -87,6 +90,15 @@ def busbw_reduce_scatter(input_bytes: float, p: int, t: float) -> float:
     return input_bytes * (p - 1) / (p * t)
 
 
+def ring_schedule_bytes(p: int, n: int, s: int) -> int:
+    """Bytes the ring's schedule moves when every message goes through device
+    memory: reduce-scatter 3(p-1) n s (each step reads the message and the
+    receiver's chunk and writes the partial, p chunks of n/p), all-gather
+    2(p-1) n s -- (5p-5) n s, 35 n s at p = 8 ("LLM Parallelism 基础", section
+    "Ring AllReduce"; the minimum is 2 p n s)."""
+    return (5 * p - 5) * n * s
+
+
 def ring_model_seconds(size_bytes: float, p: int, bw: float) -> float:
     """Ring all-reduce time model 2 (N-1)/N * S/W ("分布式训练/推理", section
     "Ring all-reduce 的带宽账")."""
@@ -114,7 +126,7 @@ KERNEL_OF = {
     "all_gather": ("rc_fanout_reg_kernel", "fanout.cu"),
     "reduce": ("rc_reduce_front_kernel", "reduce.cu"),
     "broadcast": ("rc_fanout_reg_kernel", "fanout.cu"),
-    "ring_all_reduce": ("rc_ring_chain_kernel", "ring.cu"),
+    "ring_all_reduce": ("rc_ring_link_kernel", "ring.cu"),
     "hier_all_reduce": ("rc_hier_front_kernel", "hier.cu"),
 }
 
@@ -235,6 +247,20 @@ def cpu_oracle_step_rate(budget_s: float = 12.0, n_sample: int = N // 8):
     return step_bytes * reps / el / 1e9, reps, el, n_sample
 
 
+def host_cpu():
+    """The host's logical CPU count and model name (from /proc/cpuinfo)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cpu_count": os.cpu_count(), "host_cpu_model": model}
+
+
 def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
@@ -260,7 +286,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "p": P, "n_per_rank": N, "l2": "n/a (host)"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **host_cpu()},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -328,13 +354,6 @@ def run_ours(args):
         torch.sum(clean, dim=0, out=sink)
 
     calls = calls_of(B0)
-    if args.ops:
-        keep = args.ops.split(",")
-        unknown = set(keep) - set(calls)
-        if unknown:
-            raise SystemExit(f"unknown --ops {sorted(unknown)}")
-        ops = [(nm, b) for nm, b in ops if nm in keep]
-        step_bytes = sum(b for _, b in ops)
     names = [nm for nm, _ in ops]
     K, W = args.steps, args.warmup
     # back-to-back timing: every collective is captured once into its own CUDA
@@ -600,8 +619,13 @@ def run_ours(args):
         t_rs = per_op_s["reduce_scatter"] / K
         per_op["reduce_scatter"]["busbw_gib_s"] = round(busbw_reduce_scatter(N * 4, P, t_rs) / 2**30, 1)
     if "ring_all_reduce" in per_op:
-        per_op["ring_all_reduce"]["ring_model_us_at_measured_hbm"] = round(
-            ring_model_seconds(N * 4, P, peak * 1e9) * 1e6, 2)
+        t_ring = per_op_s["ring_all_reduce"] / K
+        sched = ring_schedule_bytes(P, N, 4)
+        per_op["ring_all_reduce"].update({
+            "ring_model_us_at_measured_hbm": round(ring_model_seconds(N * 4, P, peak * 1e9) * 1e6, 2),
+            "schedule_bytes": sched,
+            "schedule_gbs": round(sched / t_ring / 1e9, 1),
+            "schedule_gbs_repeated": round(sched / rep_s["ring_all_reduce"] / 1e9, 1)})
     dom = max(names, key=lambda nm: per_op_s[nm])
     dom_b = dict(ops)[dom]
     dom_t = per_op_s[dom] / K
@@ -615,7 +639,7 @@ def run_ours(args):
         gbs, reps, el, ns = cpu_oracle_step_rate(budget_s=args.cpu_seconds)
         cpu = {"value": round(gbs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"{reps} passes of the seven-collective step on {ns} elements per rank "
-                         f"(p=8, 1/8 of the workload), one thread, {el:.1f} s"}
+                         f"(p=8, 1/8 of the workload), one thread, {el:.1f} s", **host_cpu()}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -646,6 +670,7 @@ def run_ours(args):
                      "launch_timing": ("average launch duration: CUDA events around K replays of one graph "
                                        "of 4 launches of the kernel on 4 separate input/output sets "
                                        "(4 x its inputs and outputs > L2), inside the clock-sampled region"),
+                     "frac_of_pages_8tbs": round(dom_b / dom_rep / 1e9 / PAGES_HBM_GBS, 4),
                      "achieved_split_view": round(dom_b / dom_t / 1e9, 1),
                      "frac_split_view": round(dom_b / dom_t / 1e9 / peak, 4)},
         "split_ms_per_step": round(1e3 * split_s / K, 4),
@@ -1246,6 +1271,75 @@ def run_configs(args):
     return 0
 
 
+NCU_WORKLOADS = {
+    # name: (p, n per rank, dtype, description)
+    "step": (8, 2097152, "f32", "8 ranks x 2,097,152 fp32 (8 MiB) per rank ~N(0,1e-2), the bench step's inputs"),
+    "hier_bf16": (8, 4194304, "bf16", "8 ranks (2x4) x 4,194,304 bf16 (8 MiB) per rank ~N(0,1)"),
+    "llama_eighth": (8, 202375168 // 8, "f32",
+                     "1/8 of a Llama-2-7B decoder layer: 8 ranks x 25,296,896 elements"),
+    "sweep_64mib": (8, (64 << 20) // 4, "f32", "8 ranks x 64 MiB fp32 per rank, uniform[-1,1)"),
+}
+
+
+def run_ncu_case(args):
+    """Launches for a profiler, no timing: the collective `--ncu-case` on the
+    workload `--ncu-workload`, called on S separate input/output sets in turn,
+    twice around (4 sets when a set is under 256 MiB, else 2), so that the
+    launches after the first S find the previous launch's outputs dirty in L2,
+    as a collective in a sequence does.  With ncu --cache-control none, the
+    launch numbered S (skip S) therefore counts those write-backs in its DRAM
+    traffic.  Prints one line naming the launches."""
+    import torch
+    import collective_rc_all_b200 as rc
+    op = args.ncu_case
+    p, n, dt, desc = NCU_WORKLOADS[args.ncu_workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    TT = {"f32": torch.float32, "bf16": torch.bfloat16}
+    m = n // p
+    odt = "bf16" if op in ("reduce_scatter", "all_gather") or dt == "bf16" else "f32"
+
+    def one_set():
+        d = {"x": [(torch.randn(n, generator=gen, device=dev)).to(TT[dt]) for _ in range(p)]}
+        if op == "reduce_scatter":
+            d["y"] = [torch.empty(m, dtype=TT[odt], device=dev) for _ in range(p)]
+        elif op == "all_gather":
+            d["x"] = [t[:m].to(torch.bfloat16) for t in d["x"]]
+            d["y"] = [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+        elif op == "reduce":
+            d["y"] = torch.empty(n, dtype=TT[dt], device=dev)
+        elif op == "broadcast":
+            d["y"] = [d["x"][0]] + [torch.empty(n, dtype=TT[dt], device=dev) for _ in range(p - 1)]
+        else:
+            d["y"] = [torch.empty(n, dtype=TT[dt], device=dev) for _ in range(p)]
+        return d
+
+    call = {
+        "all_reduce": lambda d: rc.rc_all_reduce(d["x"], d["y"]),
+        "reduce_scatter": lambda d: rc.rc_reduce_scatter(d["x"], d["y"], out_dtype=odt, scale=1.0 / p),
+        "all_gather": lambda d: rc.rc_all_gather(d["x"], d["y"]),
+        "reduce": lambda d: rc.rc_reduce(d["x"], d["y"], root=0),
+        "broadcast": lambda d: rc.rc_broadcast(d["x"][0], d["y"], root=0),
+        "ring_all_reduce": lambda d: rc.rc_ring_all_reduce(d["x"], d["y"], variant="literal"),
+        "hier_all_reduce": lambda d: rc.rc_hier_all_reduce(d["x"], d["y"], 4, variant="fused"),
+    }[op]
+    set_bytes = 2 * p * n * (4 if dt == "f32" else 2)
+    S = 4 if set_bytes < (256 << 20) else 2
+    sets = [one_set() for _ in range(S)]
+    torch.cuda.synchronize()
+    l0 = rc.rc_launch_count()
+    for _ in range(2):
+        for d in sets:
+            call(d)
+    torch.cuda.synchronize()
+    rc.rc_stream_status()
+    print(json.dumps({"ncu_case": op, "workload": desc, "sets": S, "calls": 2 * S,
+                      "launches": int(rc.rc_launch_count() - l0)}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1256,8 +1350,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=20.0,
                     help="total CPU budget of the reference arm (warm-up + timed steps)")
-    # profiling aids: time a subset of the step's collectives, skip side phases
-    ap.add_argument("--ops", default="", help="comma-separated subset of the step's collectives")
+    # profiling aids: skip side phases (the timed step is always the whole step)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-copy-peak", action="store_true")
     ap.add_argument("--graph", choices=["step", "per_op"], default="step",
@@ -1277,8 +1370,13 @@ def main(argv=None):
     ap.add_argument("--ddp-tokens", type=int, default=1024, help="tokens per rank of the synthetic backward")
     ap.add_argument("--zero1-elems", type=int, default=202375168,
                     help="parameters of the ZeRO-1 workload (default: one Llama-2-7B decoder layer)")
+    # launches for a profiler (no timing): one collective on one workload
+    ap.add_argument("--ncu-case", default="", choices=[""] + [nm for nm, _ in step_ops()[0]])
+    ap.add_argument("--ncu-workload", default="step", choices=sorted(NCU_WORKLOADS))
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
+    if args.ncu_case:
+        return run_ncu_case(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.sweep:

@@ -23,7 +23,7 @@ __all__ = [
     "FP32", "BF16", "INT32", "SUM", "MAX", "MIN", "RING_LITERAL", "RING_ONESHOT",
     "HIER_FUSED", "HIER_STAGED",
     "rc_all_reduce", "rc_reduce_scatter", "rc_all_gather", "rc_reduce", "rc_broadcast",
-    "rc_ring_all_reduce", "rc_ring_all_reduce_noalloc", "rc_hier_all_reduce", "rc_copy", "rc_reserve_workspace", "rc_check_buffer",
+    "rc_ring_all_reduce", "rc_ring_all_reduce_noalloc", "rc_hier_all_reduce", "rc_copy", "rc_reserve_workspace", "rc_workspace_bytes", "rc_check_buffer",
     "rc_probe_bounded_wait",
     "rc_rank_all_reduce", "rc_rank_reduce_scatter", "rc_rank_all_gather", "rc_rank_ring_step",
     "rc_ipc_handle", "rc_ipc_export", "rc_ipc_import", "rc_ipc_release",
@@ -106,6 +106,7 @@ _decl("rc_ipc_export", [_vp, _sz, ctypes.POINTER(rc_ipc_handle)])
 _decl("rc_ipc_import", [ctypes.POINTER(rc_ipc_handle), ctypes.POINTER(_vp)])
 _decl("rc_ipc_release", [_vp])
 _decl("rc_reserve_workspace", [_sz, _vp])
+_decl("rc_workspace_bytes", [ctypes.POINTER(_sz), ctypes.POINTER(_sz)])
 _decl("rc_check_buffer", [_vp, _sz])
 _decl("rc_probe_bounded_wait", [ctypes.c_uint64, _vp])
 _decl("rc_stream_status", [_vp])
@@ -442,6 +443,14 @@ def rc_probe_bounded_wait(limit_ns: int, stream=None) -> None:
 
 def rc_reserve_workspace(nbytes: int, stream=None):
     _check(lib.rc_reserve_workspace(int(nbytes), _stream(stream)), "rc_reserve_workspace")
+
+
+def rc_workspace_bytes():
+    """(live, retired): bytes of the current device's workspace block and of
+    the blocks kept alive for captured graphs."""
+    live, retired = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib.rc_workspace_bytes(ctypes.byref(live), ctypes.byref(retired)), "rc_workspace_bytes")
+    return live.value, retired.value
 
 
 def rc_stream_status(stream=None) -> int:

@@ -217,13 +217,19 @@ rc_status launched(cudaError_t e, const char *what) {
 // ---------------------------------------------------------------- workspace
 // One workspace per device.  A call on a stream other than the last user's
 // first waits for the last user's work (event), so concurrent streams never
-// share it; growth frees the old block in stream order.
+// share it; growth frees the old block in stream order.  A block that a stream
+// capture has taken is never freed before rc_finalize: the captured graph
+// keeps its address and may be replayed after the workspace has grown, so on
+// growth such a block is retired (kept allocated) instead of freed.
 struct Workspace {
   void *ptr = nullptr;
   size_t cap = 0;
   cudaStream_t last = nullptr;
   cudaEvent_t done = nullptr;
   bool used = false;
+  bool captured = false;        // a stream capture holds ptr
+  std::vector<void *> retired;  // captured blocks replaced by a larger one
+  size_t retired_bytes = 0;
 };
 std::mutex g_ws_mu;
 Workspace g_ws[kMaxDevices];
@@ -244,6 +250,7 @@ rc_status ws_acquire(size_t bytes, cudaStream_t s, void **out, int *dev_out) {
                   bytes);
     *out = w.ptr;
     *dev_out = -1;  // no event bookkeeping inside a capture
+    w.captured = true;
     return RC_OK;
   }
   if (!w.done) {
@@ -256,9 +263,15 @@ rc_status ws_acquire(size_t bytes, cudaStream_t s, void **out, int *dev_out) {
   }
   if (w.cap < bytes) {
     if (w.ptr) {
-      if ((e = cudaFreeAsync(w.ptr, s)) != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+      if (w.captured) {  // a graph may still use it: keep it until rc_finalize
+        w.retired.push_back(w.ptr);
+        w.retired_bytes += w.cap;
+      } else if ((e = cudaFreeAsync(w.ptr, s)) != cudaSuccess) {
+        return cuda_fail(e, "cudaFreeAsync");
+      }
       w.ptr = nullptr;
       w.cap = 0;
+      w.captured = false;
     }
     const size_t want = (bytes + 255) & ~(size_t)255;
     if ((e = cudaMallocAsync(&w.ptr, want, s)) != cudaSuccess) {
@@ -455,14 +468,13 @@ rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, 
     j.x[r] = send[r];
     j.y[r] = recv[r];
   }
+  if (!ring_needs_workspace(j)) return launched(launch_ring_literal(j, (cudaStream_t)stream), "ring launch");
   int dev = -1;
   const uint64_t C = (n + p - 1) / p;
   std::lock_guard<std::mutex> lock(g_ws_mu);
-  if (dt == RC_BF16) {
-    if ((st = ws_acquire(2ull * p * C * 4, (cudaStream_t)stream, &j.ws, &dev)) != RC_OK) return st;
-  }
+  if ((st = ws_acquire(2ull * p * C * 4, (cudaStream_t)stream, &j.ws, &dev)) != RC_OK) return st;
   st = launched(launch_ring_literal(j, (cudaStream_t)stream), "ring launch");
-  if (dt == RC_BF16) ws_release(dev, (cudaStream_t)stream);
+  ws_release(dev, (cudaStream_t)stream);
   return st;
 }
 
@@ -493,6 +505,7 @@ rc_status rc_ring_all_reduce_noalloc(const void *const *send, void *const *recv,
   j.dt = dt;
   j.op = op;
   j.scale = scale;
+  j.partials_in_ws = true;  // the chain kernel, bf16 partials in the fixed scratch
   for (int r = 0; r < p; ++r) {
     j.x[r] = send[r];
     j.y[r] = recv[r];
@@ -977,11 +990,26 @@ rc_status rc_finalize(void) {
     cudaSetDevice(d);
     cudaDeviceSynchronize();
     if (w.ptr && cudaFree(w.ptr) != cudaSuccess) st = fail(RC_ERR_CUDA, "cudaFree(workspace)");
+    for (void *old : w.retired)
+      if (cudaFree(old) != cudaSuccess) st = fail(RC_ERR_CUDA, "cudaFree(retired workspace)");
     if (w.done) cudaEventDestroy(w.done);
     w = Workspace{};
   }
   cudaSetDevice(cur);
+  noalloc_scratch_forget();
   return st;
+}
+
+rc_status rc_workspace_bytes(size_t *live, size_t *retired) {
+  if (!live || !retired) return fail(RC_ERR_INVALID_ARG, "output pointer is NULL");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(RC_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  *live = g_ws[dev].cap;
+  *retired = g_ws[dev].retired_bytes;
+  return RC_OK;
 }
 
 int rc_version(void) { return 100; }

@@ -64,6 +64,7 @@ struct RingJob {
   uint64_t n;
   int dt, op;
   float scale;
+  bool partials_in_ws;   // run a kernel that keeps bf16 partials in ws (chain / element form)
 };
 
 struct HierJob {
@@ -125,8 +126,11 @@ cudaError_t launch_fold_tma(const FoldJob &job, cudaStream_t s);
 cudaError_t read_and_clear_fold_timeouts(unsigned int *count);
 cudaError_t launch_fanout(const FanoutJob &job, cudaStream_t s);
 cudaError_t launch_ring_literal(const RingJob &job, cudaStream_t s);
+// Whether launch_ring_literal will read job.ws (bf16 partials in device memory).
+bool ring_needs_workspace(const RingJob &job);
 size_t noalloc_scratch_floats();
 cudaError_t noalloc_scratch_ptr(void **out);
+void noalloc_scratch_forget();  // drop the cached addresses (rc_finalize)
 cudaError_t launch_hier_fused(const HierJob &job, cudaStream_t s);
 cudaError_t launch_hier_staged(const HierJob &job, cudaStream_t s);
 cudaError_t launch_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);

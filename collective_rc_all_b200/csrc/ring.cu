@@ -30,6 +30,15 @@
 // step's x values (independent of the partials) while the current step folds:
 // only the partials' round trip through L2 stays on the dependent chain.  The
 // per-(step, rank) chunk addresses come from a table in shared memory.
+//
+// Three kernels execute this schedule:
+//  * rc_ring_link_kernel (default for 16-byte aligned buffers): the ranks are
+//    thread groups of one thread block and every message crosses a link
+//    buffer in shared memory -- a store by the sender, a block barrier, a
+//    load by the receiver.  Device memory sees x once and y once.
+//  * rc_ring_chain_kernel: the messages are partials in device memory (the
+//    receivers' y, or a workspace for bf16), one thread per chunk chain.
+//  * rc_ring_literal_kernel: element-wise form for unaligned buffers.
 #include <algorithm>
 #include <mutex>
 #include <type_traits>
@@ -466,6 +475,191 @@ cudaError_t launch_ring_chain(const RingJob &job, uint64_t C, cudaStream_t s) {
   return launch_kernel(rc_ring_chain_kernel<T, OP, CH, PF>, dim3((unsigned)grid), dim3(kChainNT), 0, s, a);
 }
 
+// ---------------------------------------------------------------------------
+// Link kernel (16-byte aligned buffers, chunks a whole number of vectors).
+//
+// One thread block owns one tile of L vector offsets [t*L, t*L + L) inside
+// every chunk, and holds all p ranks of the ring for that tile: thread group
+// r (threads r*L .. r*L + L-1) is rank r, and its thread l works on offset
+// o = t*L + l of rank r's chunks.  The ring's links are buffers in shared
+// memory: at each of the 2(p-1) steps every rank stores its message into its
+// outgoing link, the block synchronises, and every rank loads the message of
+// its predecessor from that link.  So each step is still a real send (a
+// store) and a real receive (a load) between different threads, in the
+// schedule's order, while device memory sees only the inputs, read once
+// (rank r reads x_r[chunk c][o] for every c), and the outputs, written once
+// (y_r[chunk c][o] when rank r receives finished chunk c).
+//
+// Rank r meets its own chunks in the order c_j = (r-1-j) mod p: j = 0 is the
+// chunk it sends at reduce-scatter step 0 (its own input as the message),
+// j = k+1 the chunk it receives at step k, whose partial it folds with its
+// own x (acc = msg (+) x_r, the ring order).  At step p-2 the received chunk
+// is c = r: finished, scaled and cast once, stored to y_r[chunk r].  The
+// all-gather steps then forward the finished vectors in their stored form:
+// at step k rank r sends chunk (r-k) mod p and receives chunk (r-1-k) mod p,
+// which it stores to y_r.  Partials stay in the accumulator type (fp32 for
+// fp32 and bf16, int32 for int32).  The links alternate between two buffers
+// by step parity: a link written at step s is read at step s after the
+// barrier and rewritten at step s+2, after the barrier of step s+1, by which
+// time every reader of step s is done.  One barrier per step.
+//
+// All of rank r's input loads are issued at the start, in the order of use,
+// before any of its stores: so an in-place call (y_r == x_r) reads every
+// input before the same thread overwrites it, and no other thread touches
+// x_r[.][o] or y_r[.][o].
+template <class Acc>
+__device__ __forceinline__ uint4 acc4_bits(const Acc *a) {
+  return make_uint4(acc_bits(a[0]), acc_bits(a[1]), acc_bits(a[2]), acc_bits(a[3]));
+}
+template <class Acc>
+__device__ __forceinline__ void bits_acc4(const uint4 &v, Acc *a) {
+  if constexpr (std::is_same<Acc, float>::value) {
+    a[0] = __uint_as_float(v.x); a[1] = __uint_as_float(v.y);
+    a[2] = __uint_as_float(v.z); a[3] = __uint_as_float(v.w);
+  } else {
+    a[0] = (int32_t)v.x; a[1] = (int32_t)v.y; a[2] = (int32_t)v.z; a[3] = (int32_t)v.w;
+  }
+}
+__device__ __forceinline__ uint4 ld_x_v4(const void *p) {
+  // volatile: the compiler keeps every input load ahead of the thread's
+  // first output store (in-place calls)
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+struct RingLinkParams {
+  const char *x[kMaxRanks];
+  char *y[kMaxRanks];
+  uint64_t cv;  // vectors per chunk (C / VEC)
+  uint64_t nv;  // vectors in the whole per-rank vector (n / VEC)
+  float scale;
+  int p;
+};
+
+template <class T, int OP, int PMAX, int L>
+__global__ void __launch_bounds__(PMAX * L) rc_ring_link_kernel(const __grid_constant__ RingLinkParams a) {
+  using Acc = typename T::Acc;
+  constexpr int VEC = kVec<T>;
+  constexpr int W = VEC / 4;  // 16-byte words per partial message (1, or 2 for bf16)
+  extern __shared__ uint4 link[];  // [2 parities][p senders][W][L]
+  const int p = a.p;
+  const int r = threadIdx.x / L;
+  const int l = threadIdx.x - r * L;
+  const uint64_t cv = a.cv;
+  const uint64_t o = (uint64_t)blockIdx.x * L + l;  // vector offset inside every chunk
+  auto wrap = [p](int v) { return v < 0 ? v + p : v; };  // v > -p
+  auto live = [&](int c) -> bool {  // chunk c has an element vector at offset o
+    const uint64_t b = (uint64_t)c * cv;
+    return o < cv && b + o < a.nv;
+  };
+  const int prev = wrap(r - 1);
+  pdl_wait();
+  pdl_trigger();
+
+  // rank r's inputs, chunk c_j = (r-1-j) mod p in slot j, loaded in order of use
+  uint4 xr[PMAX];
+  const char *xb = a.x[r];
+#pragma unroll
+  for (int j = 0; j < PMAX; ++j) {
+    if (j < p) {
+      const int c = wrap(r - 1 - j);
+      if (live(c)) xr[j] = ld_x_v4(xb + ((uint64_t)c * cv + o) * 16);
+    }
+  }
+  char *yb = a.y[r];
+
+  // ---- reduce-scatter: p-1 steps
+  Acc msg[VEC];
+  if (live(prev)) unpack<T>(xr[0], msg);  // step 0 sends x_r[chunk r-1]
+#pragma unroll
+  for (int k = 0; k < PMAX - 1; ++k) {
+    if (k + 1 >= p) break;
+    uint4 *out = link + ((size_t)((k & 1) * p + r) * W) * L + l;
+    const uint4 *in = link + ((size_t)((k & 1) * p + prev) * W) * L + l;
+    const int cs = wrap(r - 1 - k), cr = wrap(r - 2 - k);
+    if (live(cs)) {
+#pragma unroll
+      for (int h = 0; h < W; ++h) out[h * L] = acc4_bits(msg + 4 * h);
+    }
+    __syncthreads();
+    if (live(cr)) {
+#pragma unroll
+      for (int h = 0; h < W; ++h) bits_acc4(in[h * L], msg + 4 * h);
+      Acc xv[VEC];
+      unpack<T>(xr[k + 1], xv);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) msg[e] = combine<OP>(msg[e], xv[e]);
+    }
+  }
+  // the received chunk of the last step is r itself: finished
+  uint4 fwd = make_uint4(0, 0, 0, 0);
+  if (live(r)) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) msg[e] = finish<OP>(msg[e], a.scale);
+    char *dst = yb + ((uint64_t)r * cv + o) * 16;
+    store_out<T, VEC>(dst, msg);
+    if constexpr (std::is_same<T, BF16>::value)
+      fwd = make_uint4(pack_bf16x2(msg[0], msg[1]), pack_bf16x2(msg[2], msg[3]),
+                       pack_bf16x2(msg[4], msg[5]), pack_bf16x2(msg[6], msg[7]));
+    else
+      fwd = acc4_bits(msg);
+  }
+
+  // ---- all-gather: p-1 steps, finished vectors in their stored form
+#pragma unroll
+  for (int k = 0; k < PMAX - 1; ++k) {
+    if (k + 1 >= p) break;
+    const int par = (p - 1 + k) & 1;
+    const int cs = wrap(r - k), cr = wrap(r - 1 - k);
+    if (live(cs)) link[((size_t)(par * p + r) * W) * L + l] = fwd;
+    __syncthreads();
+    if (live(cr)) {
+      fwd = link[((size_t)(par * p + prev) * W) * L + l];
+      st_v4(yb + ((uint64_t)cr * cv + o) * 16, fwd);
+    }
+  }
+}
+
+template <class T, int OP, int PMAX, int L>
+cudaError_t launch_ring_link_t(const RingJob &job, uint64_t C, cudaStream_t s) {
+  RingLinkParams a{};
+  const int p = job.p;
+  if (p < 2 || p > PMAX) return cudaErrorInvalidValue;
+  constexpr int VEC = kVec<T>;
+  a.p = p;
+  a.cv = C / VEC;
+  a.nv = job.n / VEC;
+  a.scale = job.scale;
+  for (int r = 0; r < p; ++r) {
+    a.x[r] = static_cast<const char *>(job.x[r]);
+    a.y[r] = static_cast<char *>(job.y[r]);
+  }
+  const uint64_t grid = (a.cv + L - 1) / L;
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)2 * p * (VEC / 4) * L * 16;
+  return launch_kernel(rc_ring_link_kernel<T, OP, PMAX, L>, dim3((unsigned)grid), dim3(p * L), smem, s, a);
+}
+
+template <class T, int OP>
+cudaError_t launch_ring_link(const RingJob &job, uint64_t C, cudaStream_t s) {
+  // L = 32 lanes per rank: one warp per rank for p > 4; two warps per rank
+  // for p <= 4 keep the block at 256 threads.
+  const int lanes = env_int("RC_RING_LANES", 0);
+  if (job.p <= 4) {
+    if (lanes == 32) return launch_ring_link_t<T, OP, 4, 32>(job, C, s);
+    return launch_ring_link_t<T, OP, 4, 64>(job, C, s);
+  }
+  if (job.p <= 8) {
+    if (lanes == 64) return launch_ring_link_t<T, OP, 8, 64>(job, C, s);
+    return launch_ring_link_t<T, OP, 8, 32>(job, C, s);
+  }
+  return launch_ring_link_t<T, OP, 16, 32>(job, C, s);
+}
+
 template <class T, int OP, int PMAX>
 cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   RingParams a{};
@@ -484,7 +678,12 @@ cudaError_t run_ring(const RingJob &job, cudaStream_t s) {
   }
   constexpr int VEC = kVec<T>;
   const bool vector = aligned && a.C % VEC == 0 && a.n % VEC == 0;
-  if (vector && env_int("RC_RING_KERNEL", 1) == 1) {
+  // RC_RING_KERNEL: 2 (default) the link kernel, 1 the chain kernel, 0 the
+  // element-register kernel; a job that brings its own partial buffer
+  // (job.partials_in_ws) runs the chain kernel.
+  const int kern_sel = job.partials_in_ws ? 1 : env_int("RC_RING_KERNEL", 2);
+  if (vector && kern_sel == 2) return launch_ring_link<T, OP>(job, a.C, s);
+  if (vector && kern_sel == 1) {
     // default: 4 chains per thread, x one step ahead (72 registers, so that
     // at p = 8 every offset's chains are resident at once); measured against
     // 2 and 8 chains and a two-step prefetch.  RC_RING_KERNEL=0 selects the
@@ -541,10 +740,20 @@ size_t noalloc_scratch_floats() { return kNoallocScratchFloats; }
 
 // Device address of the array for the current device.  In host code the
 // symbol's name is only a host-side handle, so the address is looked up once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached until rc_finalize, which
+// forgets the cache (a device reset reloads the module, so it must come after
+// rc_finalize).
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptrs[64] = {};
+
+void noalloc_scratch_forget() {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  for (void *&q : g_noalloc_ptrs) q = nullptr;
+}
+
 cudaError_t noalloc_scratch_ptr(void **out) {
-  static std::mutex mu;
-  static void *ptrs[64] = {};
+  std::mutex &mu = g_noalloc_mu;
+  void **ptrs = g_noalloc_ptrs;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -558,6 +767,18 @@ cudaError_t noalloc_scratch_ptr(void **out) {
   }
   *out = ptrs[dev];
   return cudaSuccess;
+}
+
+bool ring_needs_workspace(const RingJob &job) {
+  if (job.dt != kBF16) return false;  // fp32 / int32 partials live in y
+  bool aligned = true;
+  for (int r = 0; r < job.p; ++r)
+    aligned = aligned && reinterpret_cast<uintptr_t>(job.x[r]) % 16 == 0 &&
+              reinterpret_cast<uintptr_t>(job.y[r]) % 16 == 0;
+  const uint64_t C = (job.n + job.p - 1) / job.p;
+  const bool vector = aligned && C % 8 == 0 && job.n % 8 == 0;
+  const int kern_sel = job.partials_in_ws ? 1 : env_int("RC_RING_KERNEL", 2);
+  return !(vector && kern_sel == 2);  // the link kernel keeps its partials on chip
 }
 
 cudaError_t launch_ring_literal(const RingJob &job, cudaStream_t s) {

@@ -166,10 +166,16 @@ rc_status rc_broadcast(const void *send_root, void *const *recv, int p, int root
  *  RC_RING_LITERAL executes the 2(p-1) steps: reduce-scatter step k, every
  *   rank r sends chunk (r-k-1) mod p to rank r+1, which folds it with its own
  *   chunk; all-gather step k, rank r forwards chunk (r-k) mod p to rank r+1,
- *   which overwrites.  Partials are fp32 (int32 for int32): kept in the
- *   receivers' recv buffers when dt is fp32/int32, in the library workspace
- *   (2 * p * C * 4 bytes) when dt is bf16.  One persistent launch; each thread
- *   block runs all steps on one offset range of every chunk.
+ *   which overwrites.  Partials are fp32 (int32 for int32) between steps.
+ *   One launch; each thread block runs all 2(p-1) steps on one offset range
+ *   of every chunk.  16-byte aligned buffers whose chunk length keeps that
+ *   alignment: the block's thread groups are the p ranks and each step's
+ *   messages cross link buffers in the block's shared memory (a store by the
+ *   sender, a barrier, a load by the receiver), so device memory sees every
+ *   input read once and every output written once, and no workspace is used.
+ *   Other buffers: partials are kept in the receivers' recv buffers when dt
+ *   is fp32/int32, in the library workspace (2 * p * C * 4 bytes) when dt is
+ *   bf16.
  *  RC_RING_ONESHOT reads all p ranks directly (the rc_all_reduce kernel).
  */
 rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, size_t n,
@@ -185,7 +191,9 @@ rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, 
  * device), and code running where allocation is not allowed.
  *
  * Same arguments, result bits and literal schedule as rc_ring_all_reduce with
- * RC_RING_LITERAL.  For bf16 the fp32 partials live in a fixed scratch array
+ * RC_RING_LITERAL, executed by the kernel that passes every message through
+ * device memory (partials stored by the sender and loaded by the receiver
+ * at each step).  For bf16 the fp32 partials live in a fixed scratch array
  * inside this library (16 MiB of device memory, held by every GPU that loads
  * the library until the process exits) instead of the library workspace, so
  * bf16 calls need 2 * p * ceil(n/p) <= 4,194,304; larger requests return
@@ -193,7 +201,8 @@ rc_status rc_ring_all_reduce(const void *const *send, void *const *recv, int p, 
  * their partials in recv and use no scratch.
  *  - The first call on a device looks up the scratch array's device address
  *    (once per device, that device current); make that first call before any
- *    stream capture.
+ *    stream capture.  rc_finalize forgets the looked-up addresses; a device
+ *    reset (cudaDeviceReset) must come after rc_finalize.
  *  - All calls share the one array and it keeps the last call's contents;
  *    calls whose kernels overlap on the GPU (for example on two streams) race
  *    on it.  Nothing in it needs clearing: every partial is written before it
@@ -450,9 +459,25 @@ rc_status rc_copy(const void *src, void *dst, size_t bytes, rc_stream_t stream);
  * rc_last_error).  Every collective runs this check on each buffer. */
 rc_status rc_check_buffer(const void *ptr, size_t bytes);
 
-/* Grow the workspace of (current device, stream) to at least `bytes` now, so
- * that later calls do not allocate.  Stream-ordered. */
+/* Grow the workspace of the current device to at least `bytes` now, so that
+ * later calls do not allocate (a call under stream capture cannot).
+ * Stream-ordered: the growth waits for the workspace's last user if that was
+ * another stream, and the old block is freed in `stream`'s order.  This is
+ * why it takes a stream, unlike a size-only reservation: the workspace is
+ * allocated with cudaMallocAsync, and growing it must not free a block that
+ * work still queued on another stream is using.  Pass 0 for the legacy
+ * default stream.
+ * A block that a stream capture has used is never freed before rc_finalize:
+ * the captured graph holds its address and may be replayed after a later
+ * call grew the workspace, so growth retires such a block (it stays
+ * allocated, see rc_workspace_bytes) instead of freeing it.  Call
+ * rc_finalize only when no graph that captured a call of this library will
+ * be launched again. */
 rc_status rc_reserve_workspace(size_t bytes, rc_stream_t stream);
+
+/* Bytes of the current device's workspace: *live = the block calls use now,
+ * *retired = blocks kept alive for captured graphs (freed by rc_finalize). */
+rc_status rc_workspace_bytes(size_t *live, size_t *retired);
 
 /* Synchronise `stream`, then report: RC_ERR_CUDA for an asynchronous CUDA
  * error, RC_ERR_TIMEOUT if a bounded device wait of this library gave up
@@ -475,7 +500,8 @@ const char *rc_last_error(void);
 /* Number of kernels this library has launched in this process. */
 uint64_t rc_launch_count(void);
 
-/* Free every workspace (synchronises the devices that own one). */
+/* Free every workspace, retired blocks included (synchronises the devices
+ * that own one), and forget the fixed scratch's looked-up addresses. */
 rc_status rc_finalize(void);
 
 /* Library version, major*10000 + minor*100 + patch. */

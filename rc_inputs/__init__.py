@@ -91,6 +91,25 @@ def sweep_data(p: int, n: int, seed: int, dt: str) -> List[np.ndarray]:
     return uniform(p, n, seed, dt)
 
 
+def sweep_data_device(p: int, n: int, seed: int, dt: str, device: str = "cuda") -> List[torch.Tensor]:
+    """The sweep's value distributions drawn on the device (torch's seeded
+    Philox generator for that device), for the per-rank sizes too large to
+    draw on the host in a test: floats uniform[-1, 1) (bf16: the fp32 draw
+    narrowed by torch, round-to-nearest-even), ints uniform[-2^20, 2^20).
+    Returns p device tensors (float32, bfloat16 or int32)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = []
+    for _ in range(p):
+        if dt == "i32":
+            out.append(torch.randint(-(1 << 20), 1 << 20, (n,), generator=g, device=device,
+                                     dtype=torch.int32))
+            continue
+        t = torch.rand(n, generator=g, device=device, dtype=torch.float32) * 2.0 - 1.0
+        out.append(t if dt == "f32" else t.to(torch.bfloat16))
+    return out
+
+
 def special_values(p: int, n: int, seed: int, dt: str = "f32") -> List[np.ndarray]:
     """Values that stress ordering and rounding: signed zeros, large/small
     magnitudes that cancel, exact powers of two, bf16 rounding ties."""

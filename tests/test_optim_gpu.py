@@ -135,47 +135,34 @@ def test_zero1_equals_unfused_library_chain(rc):
         assert_bits(to_host(pc[q], "bf16"), np.concatenate(want_shards), f"chain params rank {q}")
 
 
-def test_zero1_llama_layer_sampled(rc):
+def test_zero1_llama_layer_full(rc):
     """The full-size step: 8 ranks x 202,375,168 fp32 gradients ~N(0, 1e-3),
-    bf16 parameters, fp32 shards of master weights and moments; sampled
-    indices (shard boundaries included) against the oracle element by
-    element."""
+    bf16 parameters, fp32 shards of master weights and moments; every element
+    of the new state and of every rank's parameters against the oracle's
+    composition (reduce_scatter x 1/p, AdamW per shard, all_gather)."""
     p = 8
     N = rc_inputs.LLAMA2_7B_LAYER_ELEMS
-    m = N // p
     grads = rc_inputs.draw(rc_inputs.config("llama_layer_grads_f32"))
     master, ea, es = rc_inputs.draw(rc_inputs.config("zero1_state"))
-    rng = np.random.default_rng(17)
-    idx = np.unique(np.concatenate([
-        rng.integers(0, N, 100_000),
-        np.array([c * m + o for c in range(p) for o in (0, 1, 2, 7, 8, m - 9, m - 1)]),
-    ])).astype(np.int64)
-    c, j = idx // m, idx % m
-    s_master = np.array([master[a][b] for a, b in zip(c, j)], np.float32)
-    s_ea = np.array([ea[a][b] for a, b in zip(c, j)], np.float32)
-    s_es = np.array([es[a][b] for a, b in zip(c, j)], np.float32)
-    g = oracle.reduce_at(grads, idx.astype(np.uint64), "f32", "f32", "sum", 1.0 / p)
-    w_th, w_m, w_v = oracle.adamw(s_master, s_ea, s_es, g, "f32", **HP)
     gd, _ = to_dev(grads, "f32")
-    del grads
     md, _ = to_dev(master, "f32")
     ad, _ = to_dev(ea, "f32")
     sd, _ = to_dev(es, "f32")
-    del master, ea, es
     pd = [torch.empty(N, dtype=torch.bfloat16, device="cuda") for _ in range(p)]
     rc.rc_zero1_step(gd, pd, md, ad, sd, param_dtype="bf16", **HP)
     _sync(rc)
     del gd
-    ti = torch.from_numpy(idx).cuda()
-    tj, tc = torch.from_numpy(j).cuda(), torch.from_numpy(c).cuda()
-    stack = lambda ts: torch.stack(ts)[tc, tj].cpu().numpy()
-    assert_bits(stack(md), w_th, "llama zero1 master (sampled)")
-    assert_bits(stack(ad), w_m, "llama zero1 exp_avg (sampled)")
-    assert_bits(stack(sd), w_v, "llama zero1 exp_avg_sq (sampled)")
-    want_p = oracle.f32_to_bf16(w_th)
-    for q in (0, 3, p - 1):
-        got = pd[q].index_select(0, ti).view(torch.int16).cpu().numpy().view(np.uint16)
-        assert_bits(got, want_p, f"llama zero1 params rank {q} (sampled)")
+    torch.cuda.empty_cache()
+    want_p, w_th, w_m, w_v = oracle.zero1_step(grads, master, ea, es, "f32", "bf16", **HP)
+    del grads, master, ea, es
+    for r in range(p):
+        assert_bits(to_host(md[r], "f32"), w_th[r], f"llama zero1 master shard {r}")
+        assert_bits(to_host(ad[r], "f32"), w_m[r], f"llama zero1 exp_avg shard {r}")
+        assert_bits(to_host(sd[r], "f32"), w_v[r], f"llama zero1 exp_avg_sq shard {r}")
+    want = torch.from_numpy(want_p[0].view(np.int16)).cuda()
+    for q in range(p):
+        assert_bits(want_p[q], want_p[0], f"oracle params rank {q}")
+        assert torch.equal(pd[q].view(torch.int16), want), f"llama zero1 params rank {q}"
 
 
 def test_sharded_owner_broadcast_variant(rc):

@@ -3,14 +3,18 @@
 ints uniform[-2^20, 2^20)), ops sum and max, all_reduce / reduce_scatter /
 all_gather.
 
-* up to 16 MiB per rank: seeded random data, every output element compared
-  bit for bit with the CPU oracle;
-* 64 MiB .. 1 GiB per rank: integer-valued inputs x_r[i] = (i mod 1021) + r,
-  for which sum = p*(i mod 1021) + p(p-1)/2 and max = (i mod 1021) + p - 1
-  are exact in every dtype and every fold order; every element is checked
-  against that closed form (on the device, with torch);
-* one 256 MiB-per-rank random case checked against the oracle at sampled
-  indices (chunk boundaries included).
+* up to 16 MiB per rank: seeded random data drawn on the host, every output
+  element of every rank compared bit for bit with the CPU oracle;
+* 64 MiB .. 1 GiB per rank, all 12 (p, dtype) pairs: seeded random data of
+  the same distributions drawn on the device (fold-order sensitive, so the
+  ring order of "LLM Parallelism 基础", section "Ring AllReduce", decides the
+  bits), sum and max, every rank of the all-reduce and every shard of the
+  reduce-scatter compared with the oracle at 100,000 random indices plus
+  every chunk boundary +-one vector and the ragged end; the all-gather is a
+  copy and is compared in full;
+* the largest sizes also once with integer-valued inputs x_r[i] = (i mod
+  1021) + r, exact in every dtype and fold order, every element checked
+  against that closed form (on the device, with torch).
 """
 import numpy as np
 import pytest
@@ -50,8 +54,8 @@ def test_sweep_random_vs_oracle(rc, p, nbytes, dt):
         rc.rc_reduce_scatter(d, rs, op=op)
         torch.cuda.synchronize()
         rc.rc_stream_status()
-        assert_bits(to_host(y[0], dt), want[0], f"AR p={p} {nbytes}B {dt} {op} rank 0")
-        assert_bits(to_host(y[p - 1], dt), want[p - 1], f"AR p={p} {nbytes}B {dt} {op} rank p-1")
+        for r in range(p):
+            assert_bits(to_host(y[r], dt), want[r], f"AR p={p} {nbytes}B {dt} {op} rank {r}")
         assert_bits(np.concatenate([to_host(t, dt) for t in rs]), want[0],
                     f"RS p={p} {nbytes}B {dt} {op}")
     # all_gather of rank-specific shards
@@ -61,7 +65,7 @@ def test_sweep_random_vs_oracle(rc, p, nbytes, dt):
     rc.rc_all_gather(sd, ag)
     torch.cuda.synchronize()
     want_ag = np.concatenate(shards)
-    for r in (0, p - 1):
+    for r in range(p):
         assert_bits(to_host(ag[r], dt), want_ag, f"AG p={p} {nbytes}B {dt} rank {r}")
 
 
@@ -88,8 +92,8 @@ def test_sweep_large_closed_form(rc, p, nbytes, dt):
         rc.rc_all_reduce(xs, y, op=op)
         torch.cuda.synchronize()
         rc.rc_stream_status()
-        for r in (0, p - 1):
-            assert torch.equal(y[r], want), f"AR closed form p={p} {nbytes}B {dt} {op}"
+        for r in range(p):
+            assert torch.equal(y[r], want), f"AR closed form p={p} {nbytes}B {dt} {op} r{r}"
         del y
         rs = [torch.empty(n // p, dtype=TORCH[dt], device="cuda") for _ in range(p)]
         rc.rc_reduce_scatter(xs, rs, op=op)
@@ -100,30 +104,80 @@ def test_sweep_large_closed_form(rc, p, nbytes, dt):
         y = [torch.empty(n, dtype=TORCH[dt], device="cuda") for _ in range(p)]
         rc.rc_all_gather(rs, y)
         torch.cuda.synchronize()
-        for r in (0, p - 1):
-            assert torch.equal(y[r], want), f"AG closed form p={p} {nbytes}B {dt}"
+        for r in range(p):
+            assert torch.equal(y[r], want), f"AG closed form p={p} {nbytes}B {dt} r{r}"
         del y, rs, want
     del xs, base
     torch.cuda.empty_cache()
 
 
-def test_sweep_256mib_random_sampled(rc):
-    p, dt = 8, "f32"
-    n = (1 << 28) // 4
-    xs = rc_inputs.sweep_data(p, n, seed=777, dt=dt)
-    d, _ = to_dev(xs, dt)
-    y = [torch.empty(n, dtype=torch.float32, device="cuda") for _ in range(p)]
-    rc.rc_all_reduce(d, y)
-    rs = [torch.empty(n // p, dtype=torch.float32, device="cuda") for _ in range(p)]
-    rc.rc_reduce_scatter(d, rs, op="max")
+def _sample_indices(n, p, vec, seed, k=100_000):
+    """k random indices plus every chunk boundary +-vec (and +-1) and the ragged end."""
+    C = -(-n // p)
+    rng = np.random.default_rng(seed)
+    edge = []
+    for c in range(p + 1):
+        for d in (-vec, -1, 0, 1, vec):
+            if 0 <= c * C + d < n:
+                edge.append(c * C + d)
+    edge += [0, 1, n - vec, n - 2, n - 1]
+    return np.unique(np.concatenate([rng.integers(0, n, k), np.array(edge)])).astype(np.int64)
+
+
+def _sparse_host_inputs(xs, dt, idx):
+    """Host arrays of the full length n that hold the device inputs' values at
+    idx and zeros elsewhere (np.zeros maps untouched pages, so an n-element
+    array costs only the pages idx touches).  reduce_at reads x_r[idx] and
+    nothing else, so it sees exactly the inputs the GPU saw."""
+    ti = torch.from_numpy(idx).cuda()
+    out = []
+    for x in xs:
+        h = np.zeros(x.numel(), dtype={"f32": np.float32, "bf16": np.uint16, "i32": np.int32}[dt])
+        h[idx] = to_host(x.index_select(0, ti), dt)
+        out.append(h)
+    return out
+
+
+LARGE_POINTS = [(p, nbytes, dt) for nbytes in LARGE for p in (2, 4, 8, 16) for dt in ("f32", "bf16", "i32")]
+
+
+@pytest.mark.parametrize("p,nbytes,dt", LARGE_POINTS)
+def test_sweep_large_random_sampled(rc, p, nbytes, dt):
+    n = nbytes // ESZ[dt]
+    m = n // p
+    vec = 16 // ESZ[dt]
+    seed = 100 + p * 97 + nbytes % 9973
+    xs = rc_inputs.sweep_data_device(p, n, seed=seed, dt=dt)
+    idx = _sample_indices(n, p, vec, seed)
+    hx = _sparse_host_inputs(xs, dt, idx)
+    ti = torch.from_numpy(idx).cuda()
+    for op in ("sum", "max"):
+        want = oracle.reduce_at(hx, idx.astype(np.uint64), dt, dt, op)
+        y = [torch.empty(n, dtype=TORCH[dt], device="cuda") for _ in range(p)]
+        rc.rc_all_reduce(xs, y, op=op)
+        torch.cuda.synchronize()
+        rc.rc_stream_status()
+        for r in range(p):
+            assert_bits(to_host(y[r].index_select(0, ti), dt), want,
+                        f"AR p={p} {nbytes}B {dt} {op} rank {r} (sampled)")
+        del y
+        rs = [torch.empty(m, dtype=TORCH[dt], device="cuda") for _ in range(p)]
+        rc.rc_reduce_scatter(xs, rs, op=op)
+        torch.cuda.synchronize()
+        rc.rc_stream_status()
+        got = to_host(torch.cat(rs).index_select(0, ti), dt)
+        assert_bits(got, want, f"RS p={p} {nbytes}B {dt} {op} (sampled, every shard)")
+        del rs
+    # all_gather of rank-specific shards: a copy, compared in full on the device
+    shards = [x[:m] for x in xs]
+    ag = [torch.empty(n, dtype=TORCH[dt], device="cuda") for _ in range(p)]
+    rc.rc_all_gather(shards, ag)
     torch.cuda.synchronize()
     rc.rc_stream_status()
-    m = n // p
-    rng = np.random.default_rng(5)
-    idx = np.unique(np.concatenate([rng.integers(0, n, 100_000),
-                                    np.array([c * m + o for c in range(p) for o in (0, 1, 3, 4, m - 5, m - 1)])]))
-    ti = torch.from_numpy(idx.astype(np.int64)).cuda()
-    got = y[3].index_select(0, ti).cpu().numpy()
-    assert_bits(got, oracle.reduce_at(xs, idx.astype(np.uint64), dt, dt, "sum"), "AR 256MiB sampled")
-    full = torch.cat(rs).index_select(0, ti).cpu().numpy()
-    assert_bits(full, oracle.reduce_at(xs, idx.astype(np.uint64), dt, dt, "max"), "RS max 256MiB sampled")
+    want_ag = torch.cat(shards)
+    for r in range(p):
+        assert torch.equal(ag[r].view(torch.int16 if dt == "bf16" else TORCH[dt]),
+                           want_ag.view(torch.int16 if dt == "bf16" else TORCH[dt])), \
+            f"AG p={p} {nbytes}B {dt} rank {r}"
+    del ag, want_ag, shards, xs
+    torch.cuda.empty_cache()

@@ -69,3 +69,43 @@ def test_noalloc_ring_rejects_oversize_without_launch():
     st = fn(_ptrs(d), _ptrs(y), p, n, 1, 0, 1.0, torch.cuda.current_stream().cuda_stream)
     assert st == 1 and "scratch" in rc.rc_last_error()
     assert rc.rc_launch_count() == before
+
+
+def test_noalloc_ring_at_the_scratch_limit_allocates_nothing():
+    """At exactly the fixed scratch's limit (p = 8, n = 2,097,152 bf16, the
+    8 MiB-per-rank ring workload: 2*p*ceil(n/p) = 4,194,304 floats) the call
+    is accepted, gives the existing entry point's bits, and neither grows the
+    library workspace nor takes device memory; one vector more is rejected."""
+    rc, fn = _cabi()
+    stream = torch.cuda.current_stream().cuda_stream
+    p, n = 8, 2097152
+    xs = rc_inputs.normal(p, n, seed=43, sigma=1.0, dt="bf16")
+    d, _ = to_dev(xs, "bf16")
+    got, back = empty_dev(n, "bf16", p)
+    small, _ = empty_dev(64, "bf16", p)
+    assert fn(_ptrs(d), _ptrs(small), p, 64, 1, 0, 1.0, stream) == 0   # first call: address look-up
+    torch.cuda.synchronize()
+    rc.rc_finalize()                                   # no library workspace from here on
+    assert rc.rc_workspace_bytes() == (0, 0)
+    free_before = torch.cuda.mem_get_info()[0]
+    st = fn(_ptrs(d), _ptrs(got), p, n, 1, 0, 1.0, stream)
+    assert st == 0, rc.rc_last_error()
+    torch.cuda.synchronize()
+    rc.rc_stream_status()
+    assert torch.cuda.mem_get_info()[0] == free_before
+    assert rc.rc_workspace_bytes() == (0, 0)
+    want, _ = empty_dev(n, "bf16", p)
+    rc.rc_ring_all_reduce(d, want, variant="literal")
+    torch.cuda.synchronize()
+    rc.rc_stream_status()
+    for r in range(p):
+        assert_bits(to_host(got[r], "bf16"), to_host(want[r], "bf16"), f"noalloc ring at the limit r{r}")
+    for b in back:
+        assert np.all(b[n * 2:].cpu().numpy() == 0x5A)
+    n1 = n + 8                                          # ceil(n1/p) = 262,145: 16 floats too many
+    d1 = [torch.empty(n1, dtype=torch.bfloat16, device="cuda") for _ in range(p)]
+    y1 = [torch.empty(n1, dtype=torch.bfloat16, device="cuda") for _ in range(p)]
+    before = rc.rc_launch_count()
+    assert fn(_ptrs(d1), _ptrs(y1), p, n1, 1, 0, 1.0, stream) == 1
+    assert "scratch" in rc.rc_last_error()
+    assert rc.rc_launch_count() == before
