@@ -65,16 +65,36 @@ WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 
             "hierarchical all_reduce 2x4 (fused)")
 
 # DRAM traffic per launch measured by ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum) for the kernel named, together with a hash of the
-# kernel's source file when it was measured; a changed source reports null.
+# dram__bytes_write.sum) for the kernel named, with the hash of the kernel's
+# source file and the shared device helpers (common.cuh) when it was measured;
+# a changed source reports null.  Captured on the launch after a call of the
+# same collective on another buffer set, with ncu's cache control off, so the
+# previous call's dirty outputs are written back inside the captured launch
+# (bench.py --ncu-case OP --ncu-workload step).
 NCU_TRAFFIC = {
-    # op: DRAM bytes per launch (read + write, one cold-cache ncu launch of the
-    # step's workload), kernel source hash at capture time
-    "ring_all_reduce": {"bytes": 67128320 + 33989888, "src": "79d77f64a1dae252"},
-    "all_reduce": {"bytes": 67120640 + 13718528, "src": "1ed4bd8024e65e84"},
-    "reduce_scatter": {"bytes": 67119104 + 1223680, "src": "1ed4bd8024e65e84"},
-    "all_gather": {"bytes": 4200448 + 162048, "src": "222781d7ad9587f7"},
-    "hier_all_reduce": {"bytes": 67121408 + 14397184, "src": "c29ec89dde043b30"},
+    "ring_all_reduce": {"bytes": 67129088 + 64138752, "src": "c45d7fa8c7c36e21"},
+    "all_reduce": {"bytes": 67109120 + 65831168, "src": "a8286ac40f63cbac"},
+    "reduce_scatter": {"bytes": 67108864 + 5248256, "src": "a8286ac40f63cbac"},
+    "all_gather": {"bytes": 4166656 + 28433920, "src": "fc875742dd8543e5"},
+    "reduce": {"bytes": 67103488 + 9445376, "src": "a8286ac40f63cbac"},
+    "broadcast": {"bytes": 8390144 + 54746624, "src": "fc875742dd8543e5"},
+    "hier_all_reduce": {"bytes": 67109632 + 65798400, "src": "2313c768785593d6"},
+}
+
+# Each collective's duration inside the timed step graph, from one ncu
+# launch list of the timed replays (NVTX range rc_timed_step; cache control
+# off, so every kernel meets the L2 state the previous one left; mean of 3
+# steps, us) and its DRAM bytes there.  ncu serialises the launches, so the
+# absolute times run about 10% long; the bench reports each collective's
+# share of this list times the live step time.
+NCU_IN_STEP = {
+    "all_reduce": {"us": 25.43, "dram": 67.1e6 + 65.5e6, "src": "a8286ac40f63cbac"},
+    "reduce_scatter": {"us": 17.53, "dram": 67.1e6 + 14.0e6, "src": "a8286ac40f63cbac"},
+    "all_gather": {"us": 9.73, "dram": 4.2e6 + 23.3e6, "src": "fc875742dd8543e5"},
+    "reduce": {"us": 17.12, "dram": 67.1e6 + 14.1e6, "src": "a8286ac40f63cbac"},
+    "broadcast": {"us": 12.70, "dram": 8.4e6 + 46.5e6, "src": "fc875742dd8543e5"},
+    "ring_all_reduce": {"us": 26.12, "dram": 64.8e6 + 70.5e6, "src": "c45d7fa8c7c36e21"},
+    "hier_all_reduce": {"us": 25.14, "dram": 67.1e6 + 64.5e6, "src": "2313c768785593d6"},
 }
 
 
@@ -132,9 +152,13 @@ KERNEL_OF = {
 
 
 def _src_hash(fname):
-    path = os.path.join(ROOT, "collective_rc_all_b200", "csrc", fname)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel's source file plus the shared device helpers."""
+    csrc = os.path.join(ROOT, "collective_rc_all_b200", "csrc")
+    data = b""
+    for f in (fname, "common.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            data += fh.read()
+    return hashlib.sha256(data).hexdigest()[:16]
 
 
 def measured_peaks():
@@ -428,10 +452,13 @@ def run_ours(args):
     torch.cuda.synchronize()
     if step_graph is not None:
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # the NVTX range names the timed replays for a profiler's launch filter
+        torch.cuda.nvtx.range_push("rc_timed_step")
         ea.record(stream)
         for _ in range(K):
             step_graph.replay()
         eb.record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         step_s = ea.elapsed_time(eb) * 1e-3
         if world > 1:
@@ -612,6 +639,19 @@ def run_ours(args):
                       "repeated_frac_of_measured_hbm": round(b / rep_s[nm] / 1e9 / peak, 4),
                       "isolated_us": round(ti * 1e6, 2),
                       "isolated_frac_of_measured_hbm": round(b / ti / 1e9 / peak, 4)}
+    # in-step durations: each collective's share of the ncu launch list of the
+    # timed step graph, times this run's step time (null once a kernel changed)
+    ins = {nm: NCU_IN_STEP.get(nm) for nm in names}
+    if all(v is not None and v["src"] == _src_hash(KERNEL_OF[nm][1]) for nm, v in ins.items()):
+        tot_ncu = sum(v["us"] for v in ins.values())
+        for nm, b in ops:
+            t_in = ins[nm]["us"] / tot_ncu * (step_s / K)
+            per_op[nm].update({"in_step_us": round(t_in * 1e6, 2),
+                               "in_step_frac_of_measured_hbm": round(b / t_in / 1e9 / peak, 4),
+                               "in_step_ncu_us": ins[nm]["us"], "in_step_ncu_dram_bytes": int(ins[nm]["dram"])})
+    else:
+        for nm in names:
+            per_op[nm].update({"in_step_us": None, "in_step_frac_of_measured_hbm": None})
     if "all_reduce" in per_op:
         t_ar = per_op_s["all_reduce"] / K
         per_op["all_reduce"]["busbw_gib_s"] = round(busbw_all_reduce(N * 4, P, t_ar) / 2**30, 1)

@@ -9,6 +9,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -152,6 +153,33 @@ __device__ __forceinline__ void st_v4(void *p, uint4 v) {
 __device__ __forceinline__ void st_v2(void *p, uint2 v) {
   asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
+// Streaming stores (cache-streaming, .cs: the line is likely written once and
+// not read again here, so L2 evicts it first).  Used for the outputs of the
+// collectives with many destinations, which no kernel of the call reads back:
+// they leave fewer dirty lines in L2 for the next kernel to write back.
+// Measured in a sequence of seven collectives (8 ranks x 8 MiB fp32), each
+// collective back to back with itself: all-gather 8.17 -> 7.73 us, broadcast
+// 12.8 -> 12.3, hierarchical all-reduce 23.96 -> 23.56, all-reduce 24.1 ->
+// 23.8; the reduce-scatter (one small output per rank) was 3% slower with
+// them and keeps ordinary stores.
+__device__ __forceinline__ void st_v4_cs(void *p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_v2_cs(void *p, uint2 v) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+template <bool CS>
+__device__ __forceinline__ void st16(void *p, uint4 v) {
+  if constexpr (CS) st_v4_cs(p, v);
+  else st_v4(p, v);
+}
+template <bool CS>
+__device__ __forceinline__ void st8(void *p, uint2 v) {
+  if constexpr (CS) st_v2_cs(p, v);
+  else st_v2(p, v);
+}
 
 // Unpack a raw 16-byte vector of T into kVec<T> accumulators.
 template <class T>
@@ -181,34 +209,26 @@ __device__ __forceinline__ void unpack<BF16>(const uint4 &raw, float (&a)[8]) {
 }
 
 // Store VEC accumulated values (already scaled) as type TO at address p.
-// VEC * TO::kBytes is 8, 16 or 32 bytes.
-template <class TO, int VEC>
-__device__ __forceinline__ void store_vec(char *p, const typename TO::Acc (&y)[VEC]);
-
-template <>
-__device__ __forceinline__ void store_vec<F32, 4>(char *p, const float (&y)[4]) {
-  st_v4(p, make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
-                      __float_as_uint(y[3])));
-}
-template <>
-__device__ __forceinline__ void store_vec<I32, 4>(char *p, const int32_t (&y)[4]) {
-  st_v4(p, make_uint4((uint32_t)y[0], (uint32_t)y[1], (uint32_t)y[2], (uint32_t)y[3]));
-}
-template <>
-__device__ __forceinline__ void store_vec<BF16, 8>(char *p, const float (&y)[8]) {
-  st_v4(p, make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                      pack_bf16x2(y[6], y[7])));
-}
-template <>
-__device__ __forceinline__ void store_vec<BF16, 4>(char *p, const float (&y)[4]) {
-  st_v2(p, make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3])));
-}
-template <>
-__device__ __forceinline__ void store_vec<F32, 8>(char *p, const float (&y)[8]) {
-  st_v4(p, make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
-                      __float_as_uint(y[3])));
-  st_v4(p + 16, make_uint4(__float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]),
-                           __float_as_uint(y[7])));
+// VEC * TO::kBytes is 8, 16 or 32 bytes.  CS: streaming stores (st16 / st8).
+template <class TO, int VEC, bool CS = false>
+__device__ __forceinline__ void store_vec(char *p, const typename TO::Acc (&y)[VEC]) {
+  if constexpr (std::is_same<TO, F32>::value && VEC == 4) {
+    st16<CS>(p, make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                           __float_as_uint(y[3])));
+  } else if constexpr (std::is_same<TO, I32>::value && VEC == 4) {
+    st16<CS>(p, make_uint4((uint32_t)y[0], (uint32_t)y[1], (uint32_t)y[2], (uint32_t)y[3]));
+  } else if constexpr (std::is_same<TO, BF16>::value && VEC == 8) {
+    st16<CS>(p, make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                           pack_bf16x2(y[6], y[7])));
+  } else if constexpr (std::is_same<TO, BF16>::value && VEC == 4) {
+    st8<CS>(p, make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3])));
+  } else {
+    static_assert(std::is_same<TO, F32>::value && VEC == 8, "unsupported output vector");
+    st16<CS>(p, make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
+                           __float_as_uint(y[3])));
+    st16<CS>(p + 16, make_uint4(__float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]),
+                                __float_as_uint(y[7])));
+  }
 }
 
 }  // namespace rc

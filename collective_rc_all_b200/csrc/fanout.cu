@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kRegNT) rc_fanout_reg_kernel(const __grid_cons
 #pragma unroll
     for (int j = 0; j < kRegILP; ++j) {
       const uint64_t u = v0 + (uint64_t)j * kRegNT + threadIdx.x;
-      if (u < nv) st_v4(dst + u * 16, v[j]);
+      if (u < nv) st_v4_cs(dst + u * 16, v[j]);
     }
   }
 }

@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kNT) rc_hier_front_kernel(const __grid_constan
   const uint64_t off = v * VEC * (uint64_t)T::kBytes;
 #pragma unroll
   for (int r = 0; r < PMAX; ++r)
-    if (r < p) store_vec<T, VEC>(a.y[r] + off, tot);
+    if (r < p) store_vec<T, VEC, true>(a.y[r] + off, tot);
 }
 
 template <int PMAX, class T, int OP>

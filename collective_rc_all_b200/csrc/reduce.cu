@@ -149,7 +149,9 @@ __global__ void __launch_bounds__(kNT) rc_reduce_front_kernel(const __grid_const
     if (a.mode == kModeAll) {
 #pragma unroll
       for (int r = 0; r < PMAX; ++r)
-        if (r < a.ndst) store_vec<TO, VEC>(a.dst[r] + e * TO::kBytes, acc);
+        if (r < a.ndst) store_vec<TO, VEC, true>(a.dst[r] + e * TO::kBytes, acc);
+    } else if (a.mode == kModeOne) {
+      store_vec<TO, VEC, true>(d1 + e * TO::kBytes, acc);
     } else {
       store_vec<TO, VEC>(d1 + e * TO::kBytes, acc);
     }
