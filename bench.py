@@ -75,9 +75,9 @@ NCU_TRAFFIC = {
     "ring_all_reduce": {"bytes": 67129088 + 64138752, "src": "c45d7fa8c7c36e21"},
     "all_reduce": {"bytes": 67109120 + 65831168, "src": "a8286ac40f63cbac"},
     "reduce_scatter": {"bytes": 67108864 + 5248256, "src": "a8286ac40f63cbac"},
-    "all_gather": {"bytes": 4166656 + 28433920, "src": "fc875742dd8543e5"},
+    "all_gather": {"bytes": 4179200 + 28185600, "src": "0ddf8327725346c4"},
     "reduce": {"bytes": 67103488 + 9445376, "src": "a8286ac40f63cbac"},
-    "broadcast": {"bytes": 8390144 + 54746624, "src": "fc875742dd8543e5"},
+    "broadcast": {"bytes": 8397568 + 54514176, "src": "0ddf8327725346c4"},
     "hier_all_reduce": {"bytes": 67109632 + 65798400, "src": "2313c768785593d6"},
 }
 
@@ -88,13 +88,13 @@ NCU_TRAFFIC = {
 # absolute times run about 10% long; the bench reports each collective's
 # share of this list times the live step time.
 NCU_IN_STEP = {
-    "all_reduce": {"us": 25.43, "dram": 67.1e6 + 65.5e6, "src": "a8286ac40f63cbac"},
-    "reduce_scatter": {"us": 17.53, "dram": 67.1e6 + 14.0e6, "src": "a8286ac40f63cbac"},
-    "all_gather": {"us": 9.73, "dram": 4.2e6 + 23.3e6, "src": "fc875742dd8543e5"},
-    "reduce": {"us": 17.12, "dram": 67.1e6 + 14.1e6, "src": "a8286ac40f63cbac"},
-    "broadcast": {"us": 12.70, "dram": 8.4e6 + 46.5e6, "src": "fc875742dd8543e5"},
-    "ring_all_reduce": {"us": 26.12, "dram": 64.8e6 + 70.5e6, "src": "c45d7fa8c7c36e21"},
-    "hier_all_reduce": {"us": 25.14, "dram": 67.1e6 + 64.5e6, "src": "2313c768785593d6"},
+    "all_reduce": {"us": 25.54, "dram": 67.1e6 + 65.5e6, "src": "a8286ac40f63cbac"},
+    "reduce_scatter": {"us": 17.19, "dram": 67.1e6 + 13.9e6, "src": "a8286ac40f63cbac"},
+    "all_gather": {"us": 9.82, "dram": 4.2e6 + 23.3e6, "src": "0ddf8327725346c4"},
+    "reduce": {"us": 17.29, "dram": 67.1e6 + 13.8e6, "src": "a8286ac40f63cbac"},
+    "broadcast": {"us": 12.83, "dram": 8.4e6 + 47.0e6, "src": "0ddf8327725346c4"},
+    "ring_all_reduce": {"us": 25.76, "dram": 64.7e6 + 70.2e6, "src": "c45d7fa8c7c36e21"},
+    "hier_all_reduce": {"us": 25.31, "dram": 67.1e6 + 64.7e6, "src": "2313c768785593d6"},
 }
 
 
@@ -1170,7 +1170,7 @@ def run_configs(args):
     """Every named workload's calls, timed (one JSON line per call):
       uniform p=4 x 65,536 fp32         all_reduce, reduce_scatter, all_gather
       ring p=8 x 2,097,152 fp32         ring literal, ring one-shot, all_reduce
-      ring p=8 x 2,097,152 bf16         ring literal (workspace), no-allocation ring, one-shot
+      ring p=8 x 2,097,152 bf16         ring literal, no-allocation ring, one-shot
       hierarchical 2x4 x 4,194,304 bf16 fused, staged, flat all_reduce
       Llama-2-7B layer p=8              all_gather of bf16 shards, reduce_scatter
                                         fp32 -> bf16 x 1/8
@@ -1264,16 +1264,16 @@ def run_configs(args):
         emit("ring p=8 x 2,097,152 fp32", call, 2 * p * n * 4, iso(mk(S[0])), b2b([mk(d) for d in S]))
     del S
 
-    # ring p=8 x 2,097,152 bf16 (4 MiB per rank): fp32 partials in the
-    # library workspace, or in the fixed scratch of the no-allocation entry
-    # point (2 x 8 x 262,144 floats, exactly its 16 MiB)
+    # ring p=8 x 2,097,152 bf16 (4 MiB per rank): fp32 partials in the link
+    # kernel's shared memory, or (the no-allocation entry point's chain
+    # kernel) in its fixed scratch (2 x 8 x 262,144 floats, exactly 16 MiB)
     p, n = 8, 2097152
     gen.manual_seed(1)
     S = sets(4, lambda: {"x": [rand(n, "bf16", 1e-2) for _ in range(p)],
                          "y": [torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(p)]})
     rc.rc_reserve_workspace(2 * p * (n // p) * 4)
     for call, mk in (
-            ("ring_all_reduce literal (workspace)", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="literal"))),
+            ("ring_all_reduce literal", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="literal"))),
             ("ring_all_reduce_noalloc", lambda d: (lambda: rc.rc_ring_all_reduce_noalloc(d["x"], d["y"]))),
             ("ring_all_reduce one-shot", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="oneshot")))):
         emit("ring p=8 x 2,097,152 bf16", call, 2 * p * n * 2, iso(mk(S[0])), b2b([mk(d) for d in S]))
@@ -1308,6 +1308,93 @@ def run_configs(args):
     f = lambda: rc.rc_reduce_scatter(grads, out, out_dtype="bf16", scale=1.0 / p)
     emit("Llama-2-7B layer p=8", "reduce_scatter fp32->bf16 x1/8", p * N * 4 + N * 2, iso(f, 5), b2b([f], 5))
     rc.rc_stream_status()
+    return 0
+
+
+def run_pairs(args):
+    """Each collective of the step after its predecessor, timed live: for
+    every consecutive pair (X, Y) of the step's order, one CUDA graph of
+    [X, Y] on 4 separate buffer sets, and one graph of [X] on the same sets,
+    each replayed back to back; Y's in-sequence cost = T([X, Y]) - T([X])
+    per call (everything the pair adds when Y follows X, the write-back of
+    X's outputs that Y meets included).  One JSON line."""
+    import torch
+    import collective_rc_all_b200 as rc
+    import rc_inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    ops, m = step_ops()
+    xs = rc_inputs.normal(P, N, seed=SEED, sigma=SIGMA)
+    send = [torch.from_numpy(x).to(dev) for x in xs]
+
+    def buffer_set():
+        B = {k: [t.clone() for t in send] for k in ("ar", "rs", "red", "bc", "ring", "hier")}
+        B.update({"y_ar": [torch.empty(N, device=dev) for _ in range(P)],
+                  "y_ring": [torch.empty(N, device=dev) for _ in range(P)],
+                  "y_hier": [torch.empty(N, device=dev) for _ in range(P)],
+                  "y_rs": [torch.empty(m, dtype=torch.bfloat16, device=dev) for _ in range(P)],
+                  "ag_in": [torch.empty(m, dtype=torch.bfloat16, device=dev) for _ in range(P)],
+                  "y_ag": [torch.empty(N, dtype=torch.bfloat16, device=dev) for _ in range(P)],
+                  "y_red": torch.empty(N, device=dev)})
+        B["y_bc"] = [B["bc"][0]] + [torch.empty(N, device=dev) for _ in range(P - 1)]
+        rc.rc_reduce_scatter(send, B["ag_in"], out_dtype="bf16", scale=1.0 / P)
+        return B
+
+    def call(nm, B):
+        return {
+            "all_reduce": lambda: rc.rc_all_reduce(B["ar"], B["y_ar"]),
+            "reduce_scatter": lambda: rc.rc_reduce_scatter(B["rs"], B["y_rs"], out_dtype="bf16", scale=1.0 / P),
+            "all_gather": lambda: rc.rc_all_gather(B["ag_in"], B["y_ag"]),
+            "reduce": lambda: rc.rc_reduce(B["red"], B["y_red"], root=0),
+            "broadcast": lambda: rc.rc_broadcast(B["bc"][0], B["y_bc"], root=0),
+            "ring_all_reduce": lambda: rc.rc_ring_all_reduce(B["ring"], B["y_ring"], variant="literal"),
+            "hier_all_reduce": lambda: rc.rc_hier_all_reduce(B["hier"], B["y_hier"], 4, variant="fused"),
+        }[nm]
+
+    sets = [buffer_set() for _ in range(4)]
+    K = max(args.steps, 20)
+
+    def timed(seq):
+        for f in seq:
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for f in seq:
+                f()
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e-3 / (K * len(sets))
+
+    peak, _ = measured_peaks()
+    names = [nm for nm, _ in ops]
+    alg = dict(ops)
+    clocks = ClockSampler(0)
+    clocks.start()
+    single = {nm: timed([call(nm, B) for B in sets]) for nm in names}
+    rows = {}
+    for i, y in enumerate(names):
+        x = names[i - 1]  # the step's predecessor (the last op precedes the first in a sequence of steps)
+        pair = timed([f for B in sets for f in (call(x, B), call(y, B))])
+        t_y = pair - single[x]
+        rows[y] = {"after": x, "pair_us": round(pair * 1e6, 2), "after_alone_us": round(single[x] * 1e6, 2),
+                   "in_sequence_us": round(t_y * 1e6, 2), "alone_back_to_back_us": round(single[y] * 1e6, 2),
+                   "in_sequence_frac_of_measured_hbm": round(alg[y] / t_y / 1e9 / peak, 4)}
+    clk = clocks.stop()
+    rc.rc_stream_status()
+    tot = sum(r["in_sequence_us"] for r in rows.values())
+    print(json.dumps({"pairs": rows, "sum_in_sequence_us": round(tot, 2),
+                      "sum_in_sequence_gbs": round(sum(alg.values()) / tot / 1e3, 1),
+                      "peak": peak, "clocks": clk}), flush=True)
     return 0
 
 
@@ -1410,6 +1497,8 @@ def main(argv=None):
     ap.add_argument("--ddp-tokens", type=int, default=1024, help="tokens per rank of the synthetic backward")
     ap.add_argument("--zero1-elems", type=int, default=202375168,
                     help="parameters of the ZeRO-1 workload (default: one Llama-2-7B decoder layer)")
+    # each collective's live cost after its predecessor in the step
+    ap.add_argument("--pairs", action="store_true")
     # launches for a profiler (no timing): one collective on one workload
     ap.add_argument("--ncu-case", default="", choices=[""] + [nm for nm, _ in step_ops()[0]])
     ap.add_argument("--ncu-workload", default="step", choices=sorted(NCU_WORKLOADS))
@@ -1417,6 +1506,8 @@ def main(argv=None):
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     if args.ncu_case:
         return run_ncu_case(args)
+    if args.pairs:
+        return run_pairs(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.sweep:

@@ -88,6 +88,19 @@ __device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uin
                : "memory");
 }
 
+// The same with an L2 evict-first cache policy on the written lines (the
+// fan-out's outputs are written once and not read again by the kernel).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void bulk_store_hint(void *gdst, const void *smem_src, uint32_t bytes, uint64_t pol) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(gdst),
+               "r"(smem_addr(smem_src)), "r"(bytes), "l"(pol)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(32) rc_fanout_bulk_kernel(const __grid_constan
     return (uint32_t)(rem < tile ? rem : tile);
   };
 
+  const uint64_t pol = l2_policy_evict_first();
   bool failed = false;
   int64_t loads_issued = 0, loads_seen = 0;
   for (int64_t k = 0; k < K + kLookahead && !failed; ++k) {
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(32) rc_fanout_bulk_kernel(const __grid_constan
       const unsigned char *buf = smem + (size_t)s * tile;
       for (int q = 0; q < a.p; ++q) {
         if ((a.skip[q] >> r) & 1u) continue;
-        bulk_store(a.dst[q] + r * a.src_bytes + off, buf, bytes);
+        bulk_store_hint(a.dst[q] + r * a.src_bytes + off, buf, bytes, pol);
       }
       bulk_commit();
     }

@@ -275,6 +275,26 @@ def test_hier_2x4_bf16_full_size(rc):
 
 
 # ------------------------------------------------------------ ZeRO-3 layer step
+def test_llama_layer_all_gather_bulk_copy(rc, monkeypatch):
+    """The bulk-copy fan-out (RC_FANOUT_BULK=1: tiles loaded once into the
+    block's shared memory, written to every rank by bulk stores) on the
+    Llama-2-7B layer's all-gather, compared in full."""
+    monkeypatch.setenv("RC_FANOUT_BULK", "1")
+    p = 8
+    N = rc_inputs.LLAMA2_7B_LAYER_ELEMS
+    shards = rc_inputs.draw(rc_inputs.config("llama_layer_param_shards_bf16"))
+    d, _ = to_dev(shards, "bf16")
+    full, back = empty_dev(N, "bf16", p, pad_bytes=16)
+    rc.rc_all_gather(d, full)
+    _sync(rc)
+    want = torch.from_numpy(np.concatenate(shards).view(np.int16)).cuda()
+    for r in range(p):
+        assert torch.equal(full[r].view(torch.int16), want), f"bulk all_gather rank {r}"
+    check_canary(back, N * 2, fill=0x5A)
+    del full, d, want
+    torch.cuda.empty_cache()
+
+
 def test_llama_layer_zero3_collectives(rc):
     """Llama-2-7B decoder layer (202,375,168 elements), 8 ranks: all_gather of
     bf16 parameter shards, then reduce_scatter of fp32 gradients ~N(0, 1e-3)
