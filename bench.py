@@ -72,13 +72,13 @@ WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 
 # previous call's dirty outputs are written back inside the captured launch
 # (bench.py --ncu-case OP --ncu-workload step).
 NCU_TRAFFIC = {
-    "ring_all_reduce": {"bytes": 67129088 + 64138752, "src": "c45d7fa8c7c36e21"},
-    "all_reduce": {"bytes": 67109120 + 65831168, "src": "a8286ac40f63cbac"},
-    "reduce_scatter": {"bytes": 67108864 + 5248256, "src": "a8286ac40f63cbac"},
-    "all_gather": {"bytes": 4179200 + 28185600, "src": "0ddf8327725346c4"},
-    "reduce": {"bytes": 67103488 + 9445376, "src": "a8286ac40f63cbac"},
-    "broadcast": {"bytes": 8397568 + 54514176, "src": "0ddf8327725346c4"},
-    "hier_all_reduce": {"bytes": 67109632 + 65798400, "src": "2313c768785593d6"},
+    "ring_all_reduce": {"bytes": 67134208 + 63897600, "src": "209752cfdc9672f1"},
+    "all_reduce": {"bytes": 67107584 + 66091520, "src": "3194ac134632a10d"},
+    "reduce_scatter": {"bytes": 67108864 + 5088256, "src": "3194ac134632a10d"},
+    "all_gather": {"bytes": 4180224 + 28257536, "src": "02a6666765c86fcd"},
+    "reduce": {"bytes": 67109888 + 8442880, "src": "3194ac134632a10d"},
+    "broadcast": {"bytes": 8389120 + 54693888, "src": "02a6666765c86fcd"},
+    "hier_all_reduce": {"bytes": 67109632 + 65382400, "src": "5eeac14585157d2b"},
 }
 
 # Each collective's duration inside the timed step graph, from one ncu
@@ -88,13 +88,13 @@ NCU_TRAFFIC = {
 # absolute times run about 10% long; the bench reports each collective's
 # share of this list times the live step time.
 NCU_IN_STEP = {
-    "all_reduce": {"us": 25.54, "dram": 67.1e6 + 65.5e6, "src": "a8286ac40f63cbac"},
-    "reduce_scatter": {"us": 17.19, "dram": 67.1e6 + 13.9e6, "src": "a8286ac40f63cbac"},
-    "all_gather": {"us": 9.82, "dram": 4.2e6 + 23.3e6, "src": "0ddf8327725346c4"},
-    "reduce": {"us": 17.29, "dram": 67.1e6 + 13.8e6, "src": "a8286ac40f63cbac"},
-    "broadcast": {"us": 12.83, "dram": 8.4e6 + 47.0e6, "src": "0ddf8327725346c4"},
-    "ring_all_reduce": {"us": 25.76, "dram": 64.7e6 + 70.2e6, "src": "c45d7fa8c7c36e21"},
-    "hier_all_reduce": {"us": 25.31, "dram": 67.1e6 + 64.7e6, "src": "2313c768785593d6"},
+    "all_reduce": {"us": 25.98, "dram": 67.1e6 + 65.7e6, "src": "3194ac134632a10d"},
+    "reduce_scatter": {"us": 16.77, "dram": 67.1e6 + 11.5e6, "src": "3194ac134632a10d"},
+    "all_gather": {"us": 9.69, "dram": 4.2e6 + 23.5e6, "src": "02a6666765c86fcd"},
+    "reduce": {"us": 17.62, "dram": 67.1e6 + 16.9e6, "src": "3194ac134632a10d"},
+    "broadcast": {"us": 12.68, "dram": 8.4e6 + 46.5e6, "src": "02a6666765c86fcd"},
+    "ring_all_reduce": {"us": 26.08, "dram": 65.1e6 + 70.2e6, "src": "209752cfdc9672f1"},
+    "hier_all_reduce": {"us": 25.37, "dram": 67.1e6 + 64.4e6, "src": "5eeac14585157d2b"},
 }
 
 

@@ -45,7 +45,6 @@ struct A2aParams {
 
 __global__ void __launch_bounds__(kNT) rc_a2a_kernel(const __grid_constant__ A2aParams a) {
   pdl_wait();
-  pdl_trigger();
   const uint64_t t = blockIdx.x;
   // the segment holding tile t: the last s with tile0[s] <= t
   int lo = 0, hi = a.nseg - 1;

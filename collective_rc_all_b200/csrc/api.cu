@@ -63,7 +63,7 @@ int device_sm_count() {
 }
 
 bool pdl_enabled() {
-  static const bool on = env_int("RC_PDL", 0) != 0;
+  static const bool on = env_int("RC_PDL", 1) != 0;
   return on;
 }
 

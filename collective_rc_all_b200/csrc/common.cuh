@@ -23,12 +23,12 @@ constexpr int kMaxRanks = 16;
 // ---------------------------------------------------------------- dependent launch
 // See launch.cuh.  pdl_wait(): block until the kernels this grid depends on
 // have completed and their writes are visible; it must precede the first
-// global-memory access of every thread.  pdl_trigger(): this block no longer
-// holds back the launch of the next kernel in the stream.
+// global-memory access of every thread.  No kernel releases its dependents
+// early (griddepcontrol.launch_dependents): they are released as this
+// kernel's blocks exit, so the next kernel's launch overlaps only this
+// kernel's drain, and its blocks never take SM slots that this kernel's later
+// waves still need.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 // ---------------------------------------------------------------- type traits
 // Storage tags.  Each has: bytes per element, the accumulator type, and

@@ -22,7 +22,6 @@ constexpr uint64_t kBlockVecs = (uint64_t)kNT * kILP;  // 16 KiB per block
 __global__ void __launch_bounds__(kNT) rc_copy_kernel(const char *__restrict__ src,
                                                       char *__restrict__ dst, uint64_t nvec) {
   pdl_wait();
-  pdl_trigger();
   const uint64_t base = (uint64_t)blockIdx.x * kBlockVecs;
   uint4 v[kILP];
 #pragma unroll
@@ -39,7 +38,6 @@ __global__ void __launch_bounds__(kNT) rc_copy_kernel(const char *__restrict__ s
 
 __global__ void rc_copy_bytes_kernel(const unsigned char *src, unsigned char *dst, uint64_t n) {
   pdl_wait();
-  pdl_trigger();
   for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n;
        i += (uint64_t)gridDim.x * blockDim.x)
     dst[i] = src[i];

@@ -64,7 +64,6 @@ __global__ void __launch_bounds__(32) rc_fanout_bulk_kernel(const __grid_constan
   for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
   mbar_init_fence();
   pdl_wait();
-  pdl_trigger();
 
   const uint64_t G = gridDim.x;
   const uint64_t u0 = a.units * blockIdx.x / G;
@@ -132,7 +131,6 @@ template <int kRegILP>
 __global__ void __launch_bounds__(kRegNT) rc_fanout_reg_kernel(const __grid_constant__ FanoutParams a,
                                                                uint64_t tiles_per_src) {
   pdl_wait();
-  pdl_trigger();
   const uint64_t r = blockIdx.x / tiles_per_src;
   const uint64_t v0 = (blockIdx.x - r * tiles_per_src) * (uint64_t)(kRegNT * kRegILP);
   const uint64_t nv = a.src_bytes / 16;
@@ -160,7 +158,6 @@ __global__ void __launch_bounds__(kRegNT) rc_fanout_reg_kernel(const __grid_cons
 template <typename E>
 __global__ void rc_fanout_elem_kernel(const __grid_constant__ FanoutParams a, int nsrc) {
   pdl_wait();
-  pdl_trigger();
   const int q = blockIdx.y;
   const uint64_t per_src = a.src_bytes / sizeof(E);
   const uint64_t total = per_src * nsrc;

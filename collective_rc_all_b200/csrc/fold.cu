@@ -147,7 +147,6 @@ __global__ void __launch_bounds__(kFoldNT, 1) rc_fold_tma_kernel(const __grid_co
   }
   __syncthreads();
   pdl_wait();
-  pdl_trigger();
 
   const uint64_t Gd = gridDim.x;
   const int64_t K = a.ntiles > blockIdx.x ? (int64_t)((a.ntiles - blockIdx.x + Gd - 1) / Gd) : 0;

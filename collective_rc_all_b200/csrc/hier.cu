@@ -45,7 +45,6 @@ __global__ void __launch_bounds__(kNT) rc_hier_reg_kernel(const __grid_constant_
   constexpr int VEC = VECTOR ? kVec<T> : 1;
   const int p = a.p, G = a.G, ng = a.ng;
   pdl_wait();
-  pdl_trigger();
   const uint64_t Gd = gridDim.x;
   uint64_t u0 = a.units * blockIdx.x / Gd;
   const uint64_t u1 = a.units * (blockIdx.x + 1) / Gd;
@@ -129,7 +128,6 @@ __global__ void __launch_bounds__(kNT) rc_hier_front_kernel(const __grid_constan
   using Acc = typename T::Acc;
   constexpr int VEC = kVec<T>;
   pdl_wait();
-  pdl_trigger();
   const int p = a.p, ng = a.ng;
   const uint64_t sg = blockIdx.x / tiles_per_seg;
   const uint64_t v0 = sg * seg_vecs + (blockIdx.x - sg * tiles_per_seg) * (uint64_t)kNT;

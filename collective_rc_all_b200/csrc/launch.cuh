@@ -1,25 +1,28 @@
 // launch.cuh -- how every kernel of this library is launched.
 //
-// Kernels can go out with programmatic dependent launch: the launch carries the
-// programmatic stream-serialization attribute, so the GPU may schedule the
-// kernel's thread blocks while the previous kernel in the stream is still
-// draining, and each kernel triggers its own dependents as soon as all of its
-// blocks are running.  The contract that keeps this exact: every kernel runs
-// pdl_wait() (griddepcontrol.wait) before its first global-memory access.
-// That instruction returns once the kernels it depends on have completed and
+// Kernels go out with programmatic dependent launch: the launch carries the
+// programmatic stream-serialization attribute, so the GPU may launch a
+// kernel while the previous kernel in the stream is still completing.  The
+// contract that keeps this exact: every kernel runs pdl_wait()
+// (griddepcontrol.wait) before its first global-memory access.  That
+// instruction returns once the kernels it depends on have completed and
 // their memory operations are visible, so a kernel reads and writes global
 // memory only after everything earlier in the stream is finished, exactly as
-// with an ordinary launch; only the launch latency and the kernel's prologue
-// (shared-memory tables, mbarrier set-up) overlap the previous kernel's tail.
-// Stream capture turns the attribute into programmatic graph edges.
+// with an ordinary launch; only the launch itself and the kernel's prologue
+// (index arithmetic, shared-memory set-up) overlap the previous kernel's
+// drain.  No kernel triggers its dependents early: they are released as its
+// blocks exit.  Stream capture turns the attribute into programmatic graph
+// edges.
 //
-// Off by default: RC_PDL=1 in the environment (read once per process) turns
-// it on.  Measured on a sequence of seven different collectives captured in
-// one graph, it changed nothing with the bulk-copy fan-out (133.8 vs 133.5 us)
-// and cost 5% with the register fan-out (138.8 vs 131.1 us), presumably
-// because the dependents' blocks, resident early and waiting at
-// griddepcontrol.wait, take issue slots from the running kernel.  Without
-// the attribute griddepcontrol.wait returns at once.
+// Measured on the sequence of seven collectives captured in one graph
+// (8 ranks x 8 MiB fp32): 117.0 us per step against 120.4 us with ordinary
+// launches, and every collective faster back to back with itself (ring
+// 23.67 -> 23.16 us, reduce-scatter 12.32 -> 11.80, all-gather 7.74 ->
+// 7.55).  With each block releasing its dependents at its start instead, the
+// dependents' blocks became resident early and took issue slots and SM room
+// from the running kernel's later waves: 121.4 against 121.0 us, and 5%
+// slower with the register fan-out.  RC_PDL=0 in the environment (read once
+// per process) turns the attribute off.
 #pragma once
 
 #include <cuda_runtime.h>

@@ -116,7 +116,6 @@ __global__ void __launch_bounds__(kNT) rc_zero1_front_kernel(const __grid_consta
                                                              uint64_t tiles_per_shard) {
   constexpr int VEC = kVec<TG>;
   pdl_wait();
-  pdl_trigger();
   const int p = a.p;
   const uint64_t mvec = a.m / VEC;
   const uint64_t c = blockIdx.x / tiles_per_shard;
@@ -179,7 +178,6 @@ __global__ void __launch_bounds__(kNT) rc_zero1_front_kernel(const __grid_consta
 template <int PMAX, class TG, class TP>
 __global__ void __launch_bounds__(kNT) rc_zero1_elem_kernel(const __grid_constant__ Zero1Params a) {
   pdl_wait();
-  pdl_trigger();
   const int p = a.p;
   for (uint64_t i = blockIdx.x * (uint64_t)kNT + threadIdx.x; i < a.n; i += (uint64_t)gridDim.x * kNT) {
     const uint64_t c = i / a.m, j = i - c * a.m;
@@ -208,7 +206,6 @@ template <class TG>
 __global__ void __launch_bounds__(kNT) rc_adamw_kernel(const __grid_constant__ AdamwParams a) {
   constexpr int VEC = kVec<TG>;
   pdl_wait();
-  pdl_trigger();
   const uint64_t stride = (uint64_t)gridDim.x * kNT;
   uint64_t done = 0;
   if (a.vector) {

@@ -57,7 +57,6 @@ __global__ void __launch_bounds__(kStepNT) rc_rank_ring_step_kernel(const __grid
   constexpr int VEC = kVec<T>;
   constexpr int PW = VEC / 4;  // 16-byte words of a vector's partial
   pdl_wait();
-  pdl_trigger();
   for (uint64_t u = blockIdx.x * (uint64_t)kStepNT + threadIdx.x; u < a.units;
        u += (uint64_t)gridDim.x * kStepNT) {
     Acc acc[VEC];
@@ -98,7 +97,6 @@ __global__ void __launch_bounds__(kStepNT) rc_rank_ring_step_scalar_kernel(const
   using Acc = typename T::Acc;
   using P = PartialOf<T>;
   pdl_wait();
-  pdl_trigger();
   for (uint64_t e = blockIdx.x * (uint64_t)kStepNT + threadIdx.x; e < a.len; e += (uint64_t)gridDim.x * kStepNT) {
     Acc acc = a.first ? load_elem<T>(a.msg, e) : (Acc)load_elem<P>(a.msg, e);
     acc = combine<OP>(acc, load_elem<T>(a.own, e));

@@ -62,7 +62,6 @@ template <int PMAX, class TI, class TO, int OP>
 __global__ void __launch_bounds__(kNT) rc_reduce_scalar_kernel(const __grid_constant__ ReduceParams a) {
   using Acc = typename TI::Acc;
   pdl_wait();
-  pdl_trigger();
   const int p = a.p;
   const uint64_t G = gridDim.x;
   // a.nvec elements starting at element c0 * C (the launch's chunk range)
@@ -102,7 +101,6 @@ __global__ void __launch_bounds__(kNT) rc_reduce_front_kernel(const __grid_const
                                                               uint64_t tiles_per_chunk) {
   using Acc = typename TI::Acc;
   pdl_wait();
-  pdl_trigger();
   constexpr int VEC = kVec<TI>;
   const int p = a.p;
   const uint64_t cvec = a.C / VEC;
@@ -165,7 +163,6 @@ __global__ void __launch_bounds__(32) rc_reduce_tail_kernel(const __grid_constan
                                                           uint64_t first, uint64_t last) {
   using Acc = typename TI::Acc;
   pdl_wait();
-  pdl_trigger();
   const int p = a.p;
   for (uint64_t e = first + threadIdx.x; e < last; e += blockDim.x) {
     const uint64_t c = e / a.C;

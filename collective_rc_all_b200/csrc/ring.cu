@@ -241,7 +241,6 @@ __global__ void __launch_bounds__(kRingNT, (PMAX <= 8 ? 4 : 2))
   }
   __syncthreads();
   pdl_wait();
-  pdl_trigger();
 
   const uint64_t G = gridDim.x;
   const uint64_t o0 = a.units * blockIdx.x / G;
@@ -367,7 +366,6 @@ __global__ void __launch_bounds__(kChainNT) rc_ring_chain_kernel(const __grid_co
   constexpr int kIn = T::kBytes;
   constexpr bool kWs = std::is_same<T, BF16>::value;
   pdl_wait();
-  pdl_trigger();
   const int p = a.p;
   const uint64_t tile = blockIdx.x / (uint32_t)a.ngroups;
   const int grp = (int)(blockIdx.x - tile * (uint32_t)a.ngroups);
@@ -591,7 +589,6 @@ __global__ void __launch_bounds__(PMAX * L, MINB) rc_ring_link_kernel(const __gr
   };
   const int prev = wrap(r - 1);
   pdl_wait();
-  pdl_trigger();
 
   // rank r's inputs, chunk c_j = (r-1-j) mod p in slot j, loaded in order of
   // use: into registers, or (XS) by asynchronous copies into shared memory,
