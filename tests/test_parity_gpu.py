@@ -154,7 +154,16 @@ def test_identity_all_reduce_equals_rs_plus_ag(rc):
 
 
 # ------------------------------------------------------------ literal ring
-RING_KERNELS = {"link": "2", "chain": "1", "element": "0"}
+# RC_RING_KERNEL value and RC_RING_XSMEM value of each ring kernel: the link
+# kernel with its inputs staged in shared memory (default) or held in
+# registers, the chain kernel, the element kernel
+RING_KERNELS = {"link": ("2", "1"), "link_regs": ("2", "0"), "chain": ("1", "1"), "element": ("0", "1")}
+
+
+def _ring_kernel(monkeypatch, kernel):
+    k, xs = RING_KERNELS[kernel]
+    monkeypatch.setenv("RC_RING_KERNEL", k)
+    monkeypatch.setenv("RC_RING_XSMEM", xs)
 
 
 @pytest.mark.parametrize("p,n", [(2, 64), (3, 1001), (3, 840), (4, 65536), (5, 12), (8, 8 * 1024 + 24),
@@ -166,7 +175,7 @@ def test_ring_literal(rc, p, n, dt, kernel, monkeypatch):
     RC_RING_KERNEL; aligned vector paths where the chunk length allows,
     element-wise otherwise): ragged chunks ((12, 760): a short last chunk;
     (16, 120): an empty one), several tiles with a ragged last tile."""
-    monkeypatch.setenv("RC_RING_KERNEL", RING_KERNELS[kernel])
+    _ring_kernel(monkeypatch, kernel)
     xs = _data(p, n, dt, seed=3000 + p + n)
     d, _ = to_dev(xs, dt)
     for op in OPS:
@@ -217,7 +226,7 @@ def test_ring_bf16_p8_8mib_full_size(rc):
 
 @pytest.mark.parametrize("kernel", sorted(RING_KERNELS))
 def test_ring_in_place(rc, kernel, monkeypatch):
-    monkeypatch.setenv("RC_RING_KERNEL", RING_KERNELS[kernel])
+    _ring_kernel(monkeypatch, kernel)
     p, n = 8, 8 * 4096
     for dt in DTS:
         xs = _data(p, n, dt, seed=77)
@@ -630,3 +639,39 @@ def test_workspace_kept_for_a_captured_graph(rc):
     torch.cuda.synchronize()
     rc.rc_finalize()
     assert rc.rc_workspace_bytes() == (0, 0)
+
+
+def test_ordinary_launches_match_oracle():
+    """With programmatic dependent launch turned off (RC_PDL=0, read once per
+    process, so in a child process) every collective of the bench step still
+    gives the oracle's bits, launched back to back on one stream."""
+    import os
+    import subprocess
+    import sys
+    code = r"""
+import numpy as np, torch, sys
+sys.path.insert(0, %r)
+sys.path.insert(0, %r)
+import collective_rc_all_b200 as rc, oracle, rc_inputs
+from util import to_dev, empty_dev, to_host, assert_bits
+p, n = 8, 8 * 4096
+xs = rc_inputs.normal(p, n, seed=61, sigma=1.0)
+d, _ = to_dev(xs, "f32")
+y, _ = empty_dev(n, "f32", p); rs, _ = empty_dev(n // p, "bf16", p); ag, _ = empty_dev(n, "bf16", p)
+ring, _ = empty_dev(n, "f32", p); h, _ = empty_dev(n, "f32", p)
+rc.rc_all_reduce(d, y); rc.rc_reduce_scatter(d, rs, out_dtype="bf16", scale=1.0 / p)
+rc.rc_all_gather(rs, ag); rc.rc_ring_all_reduce(d, ring); rc.rc_hier_all_reduce(d, h, 4)
+torch.cuda.synchronize(); rc.rc_stream_status()
+want = oracle.all_reduce(xs); want_rs = oracle.reduce_scatter(xs, "f32", "bf16", "sum", 1.0 / p)
+want_h = oracle.hier_all_reduce(xs, 4)
+for r in range(p):
+    assert_bits(to_host(y[r], "f32"), want[r], "all_reduce")
+    assert_bits(to_host(ring[r], "f32"), want[r], "ring")
+    assert_bits(to_host(h[r], "f32"), want_h[r], "hier")
+    assert_bits(to_host(rs[r], "bf16"), want_rs[r], "reduce_scatter")
+    assert_bits(to_host(ag[r], "bf16"), np.concatenate(want_rs), "all_gather")
+print("ok")
+""" % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))), os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RC_PDL="0")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
