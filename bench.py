@@ -419,6 +419,7 @@ def run_ours(args):
 
     # copy roofline of this library's own copy kernel (same run), 1 GiB
     copy_gbs = None
+    copy_same_us = None
     if not args.no_copy_peak:
         cp_a = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
         cp_b = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
@@ -435,6 +436,30 @@ def run_ours(args):
             cps.append(a.elapsed_time(b) * 1e-3)
         copy_gbs = 2 * (1 << 30) / min(cps) / 1e9
         del cp_a, cp_b
+        # the same copy kernel moving exactly an all-reduce's algorithmic
+        # bytes (64 MiB read + 64 MiB written), back to back on 4 separate
+        # buffer pairs in one graph: the size-matched ceiling the 8 MiB-per-
+        # rank collectives' back-to-back times compare with
+        half = P * N * 4
+        pairs = [(torch.empty(half, dtype=torch.uint8, device=dev),
+                  torch.empty(half, dtype=torch.uint8, device=dev)) for _ in range(4)]
+        for a_, b_ in pairs:
+            rc.rc_copy(a_, b_)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for a_, b_ in pairs:
+                rc.rc_copy(a_, b_)
+        for _ in range(3):
+            g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+        copy_same_us = a.elapsed_time(b) * 1e-3 / (4 * K) * 1e6
+        del g, pairs
 
     # the clock sampler starts before the warm-up, so the GPU is busy (not
     # idling at low clocks) when the timed region begins
@@ -716,6 +741,12 @@ def run_ours(args):
         "split_ms_per_step": round(1e3 * split_s / K, 4),
         "per_op": per_op,
         "copy_kernel_gbs": round(copy_gbs, 1) if copy_gbs else None,
+        "copy_134MB_back_to_back": ({"us": round(copy_same_us, 2),
+                                     "gbs": round(2 * P * N * 4 / copy_same_us / 1e3, 1),
+                                     "what": "this library's copy kernel moving 64 MiB -> 64 MiB (an 8 x 8 MiB "
+                                             "all-reduce's algorithmic bytes), 4 buffer pairs in one graph, "
+                                             "replayed back to back"}
+                                    if copy_same_us else None),
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": int(launches),
