@@ -675,3 +675,44 @@ print("ok")
     env = dict(os.environ, RC_PDL="0")
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("p,n", [(12, 760), (16, 120), (3, 840)])
+def test_link_ring_in_place_ragged(rc, p, n):
+    """The link kernel in place with ragged chunks (a short or an empty last
+    chunk): every input is read before its thread's first store."""
+    for dt in DTS:
+        if dt == "bf16" and (-(-n // p)) % 8:
+            continue   # the chunk length must keep 16-byte vectors for the link kernel
+        xs = _data(p, n, dt, seed=p + n)
+        want = oracle.ring_all_reduce(xs, dt)
+        d, _ = to_dev(xs, dt)
+        rc.rc_ring_all_reduce(d, d)
+        _sync(rc)
+        for r in range(p):
+            assert_bits(to_host(d[r], dt), want[r], f"link ring in place p={p} n={n} {dt} r{r}")
+
+
+def test_link_ring_captures_without_workspace(rc):
+    """The default bf16 literal ring keeps its partials on chip: it can be
+    captured into a CUDA graph with no library workspace reserved, allocates
+    none, and replays to the oracle's bits."""
+    p, n = 8, 8 * 4096
+    xs = rc_inputs.normal(p, n, seed=71, sigma=1.0, dt="bf16")
+    want = oracle.ring_all_reduce(xs, "bf16")
+    d, _ = to_dev(xs, "bf16")
+    y, _ = empty_dev(n, "bf16", p)
+    torch.cuda.synchronize()
+    rc.rc_finalize()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            rc.rc_ring_all_reduce(d, y)
+        g.replay()
+    s.synchronize()
+    rc.rc_stream_status(s)
+    assert rc.rc_workspace_bytes() == (0, 0)
+    for r in range(p):
+        assert_bits(to_host(y[r], "bf16"), want[r], f"captured bf16 ring r{r}")
+    del g
