@@ -1202,6 +1202,7 @@ def run_configs(args):
       uniform p=4 x 65,536 fp32         all_reduce, reduce_scatter, all_gather
       ring p=8 x 2,097,152 fp32         ring literal, ring one-shot, all_reduce
       ring p=8 x 2,097,152 bf16         ring literal, no-allocation ring, one-shot
+      ring p in {2, 4, 16}, 8 MiB/rank  ring literal, one-shot (fp32 and bf16)
       hierarchical 2x4 x 4,194,304 bf16 fused, staged, flat all_reduce
       Llama-2-7B layer p=8              all_gather of bf16 shards, reduce_scatter
                                         fp32 -> bf16 x 1/8
@@ -1309,6 +1310,21 @@ def run_configs(args):
             ("ring_all_reduce one-shot", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="oneshot")))):
         emit("ring p=8 x 2,097,152 bf16", call, 2 * p * n * 2, iso(mk(S[0])), b2b([mk(d) for d in S]))
     del S
+
+    # the literal ring against the one-shot across p, 8 MiB per rank
+    for p in (2, 4, 16):
+        for dt in ("f32", "bf16"):
+            n = (8 << 20) // (4 if dt == "f32" else 2)
+            gen.manual_seed(1)
+            S = sets(4, lambda: {"x": [rand(n, dt, 1e-2) for _ in range(p)],
+                                 "y": [torch.empty(n, dtype=TT[dt], device=dev) for _ in range(p)]})
+            for call, mk in (
+                    ("ring_all_reduce literal", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="literal"))),
+                    ("ring_all_reduce one-shot", lambda d: (lambda: rc.rc_ring_all_reduce(d["x"], d["y"], variant="oneshot")))):
+                emit(f"ring p={p} x {n:,} {'fp32' if dt == 'f32' else 'bf16'}", call, 2 * p * n * (4 if dt == "f32" else 2),
+                     iso(mk(S[0])), b2b([mk(d) for d in S]))
+            del S
+    torch.cuda.empty_cache()
 
     # hierarchical 2 x 4 x 4,194,304 bf16 N(0, 1)
     p, n = 8, 4194304
