@@ -1217,7 +1217,7 @@ def run_configs(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    peak, _ = measured_peaks()
+    peak, peak_kind = measured_peaks()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.ones(CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -1267,7 +1267,8 @@ def run_configs(args):
                "isolated_us": round(t_iso * 1e6, 2), "isolated_gbs": round(byt / t_iso / 1e9, 1),
                "isolated_frac_of_measured_hbm": round(byt / t_iso / 1e9 / peak, 4),
                "back_to_back_us": round(t_b2b * 1e6, 2), "back_to_back_gbs": round(byt / t_b2b / 1e9, 1),
-               "back_to_back_frac_of_measured_hbm": round(byt / t_b2b / 1e9 / peak, 4)}
+               "back_to_back_frac_of_measured_hbm": round(byt / t_b2b / 1e9 / peak, 4),
+               "peak_gbs": peak, "peak_kind": peak_kind}
         print(json.dumps(row), flush=True)
 
     def sets(k, make):
