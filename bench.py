@@ -524,6 +524,32 @@ def run_ours(args):
         b.synchronize()
         rep_s[nm] = a.elapsed_time(b) * 1e-3 / (K * len(fs))
         del g
+    # in sequence: each collective after its predecessor in the step (the
+    # last one precedes the first in a sequence of steps), live: one graph of
+    # [X, Y] on each of the 4 sets, replayed K times, minus the repeated view
+    # of X alone (the same 4 sets) -- what Y adds when it follows X
+    seq_s = {}
+    for i, y in enumerate(names):
+        x = names[i - 1]
+        fs = [f for Bx in rep_sets for f in (calls_of(Bx)[x], calls_of(Bx)[y])]
+        for f in fs:
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            for f in fs:
+                f()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+        seq_s[y] = (x, a.elapsed_time(b) * 1e-3 / (K * len(rep_sets)) - rep_s[x])
+        del g
     del rep_sets
     time.sleep(0.3)
     clk = clocks.stop()
@@ -661,6 +687,9 @@ def run_ours(args):
                       "frac_of_measured_hbm": round(b / t / 1e9 / peak, 4),
                       "frac_of_copy_kernel": round(b / t / 1e9 / copy_gbs, 4) if copy_gbs else None,
                       "repeated_us": round(rep_s[nm] * 1e6, 2),
+                      "in_sequence_after": seq_s[nm][0],
+                      "in_sequence_us": round(seq_s[nm][1] * 1e6, 2),
+                      "in_sequence_frac_of_measured_hbm": round(b / seq_s[nm][1] / 1e9 / peak, 4),
                       "repeated_frac_of_measured_hbm": round(b / rep_s[nm] / 1e9 / peak, 4),
                       "isolated_us": round(ti * 1e6, 2),
                       "isolated_frac_of_measured_hbm": round(b / ti / 1e9 / peak, 4)}
