@@ -790,7 +790,8 @@ def run_sweep(args):
     """The sweep configuration: p in {2,4,8,16}, per-rank sizes 1 KiB .. max in
     powers of 4, fp32/bf16/int32, all_reduce and reduce_scatter with sum and
     max, all_gather.  One JSON line per point: single-call device time (L2
-    flushed before every call, outside the events), effective GB/s on the
+    flushed before every call, outside the events; median and min of 200
+    calls below 1 MiB per rank, 20 up to 64 MiB, 5 above), effective GB/s on the
     minimum-bytes basis, and for sizes <= 4 MiB the per-call time inside a
     CUDA graph of 20 back-to-back calls (the launch-latency term)."""
     import torch
@@ -865,7 +866,7 @@ def run_sweep(args):
                     ("reduce_scatter", "max", lambda: rc.rc_reduce_scatter(send, rs, op="max"), p * n * s + n * s),
                     ("all_gather", "-", lambda: rc.rc_all_gather(rs, y), n * s + p * n * s),
                 ]
-                reps = 20 if nbytes <= (64 << 20) else 5
+                reps = 200 if nbytes < (1 << 20) else (20 if nbytes <= (64 << 20) else 5)
                 for coll, op, fn, byt in cases:
                     med, mn = time_call(fn, byt, reps)
                     row = {"p": p, "bytes_per_rank": nbytes, "dtype": dt, "coll": coll, "op": op,
