@@ -513,6 +513,10 @@ cudaError_t launch_ring_chain(const RingJob &job, uint64_t C, cudaStream_t s) {
 // first store follows the wait for the last slot), so an in-place call
 // (y_r == x_r) is safe, and no other thread touches x_r[.][o] or y_r[.][o].
 //
+// At p > 8 only a window of 4 slots per thread is staged (slot j + 4 is
+// requested into slot j's buffer once slot j is consumed), so that blocks of
+// 16 ranks still fit several to an SM.
+//
 // Lanes per rank: 16 for p > 4 (128-thread blocks at p = 8), 32 for p <= 4:
 // measured at p = 8, 16 lanes gave 25.2 us against 25.6 for 32 and 27.3 for
 // 64 (inputs in registers).
@@ -569,7 +573,7 @@ struct RingLinkParams {
   int p;
 };
 
-template <class T, int OP, int PMAX, int L, int MINB, bool XS>
+template <class T, int OP, int PMAX, int L, int MINB, bool XS, int XD = 0>
 __global__ void __launch_bounds__(PMAX * L, MINB) rc_ring_link_kernel(const __grid_constant__ RingLinkParams a) {
   using Acc = typename T::Acc;
   constexpr int VEC = kVec<T>;
@@ -594,33 +598,45 @@ __global__ void __launch_bounds__(PMAX * L, MINB) rc_ring_link_kernel(const __gr
   // use: into registers, or (XS) by asynchronous copies into shared memory,
   // one commit group per slot (PMAX groups, the ones past p empty), so that
   // slot j is ready once at most PMAX-1-j groups are pending
+  // With a window (XD > 0) only XD slots per thread exist: slot j lives in
+  // buffer j % XD, slot j + XD is requested as soon as slot j has been
+  // consumed, and every wait allows XD - 1 pending groups.
+  constexpr int NS = (XS && XD > 0) ? XD : PMAX;  // staged slots per thread
   uint4 xr[XS ? 1 : PMAX];
-  uint4 *xs = link + (size_t)2 * p * W * L + (size_t)r * p * L + l;  // slot j at xs[j * L]
+  uint4 *xs = link + (size_t)2 * p * W * L + (size_t)r * (XD > 0 ? XD : p) * L + l;
   const char *xb = a.x[r];
-#pragma unroll
-  for (int j = 0; j < PMAX; ++j) {
+  auto request = [&](int j) {  // slot j (one commit group, empty past p or off the data)
     if (j < p) {
       const int c = wrap(r - 1 - j);
       if (live(c)) {
-        if constexpr (XS) cp_async16(xs + j * L, xb + ((uint64_t)c * cv + o) * 16);
+        if constexpr (XS) cp_async16(xs + (j % NS) * L, xb + ((uint64_t)c * cv + o) * 16);
         else xr[j] = ld_x_v4(xb + ((uint64_t)c * cv + o) * 16);
       }
     }
     if constexpr (XS) cp_async_commit();
-  }
+  };
+#pragma unroll
+  for (int j = 0; j < NS; ++j) request(j);
   auto xslot = [&](int j) -> uint4 {
-    if constexpr (XS) {
+    if constexpr (XS && XD > 0) {
+      cp_async_wait<XD - 1>();
+      return xs[(j % NS) * L];
+    } else if constexpr (XS) {
       cp_async_wait_rt<PMAX>(PMAX - 1 - j);
       return xs[j * L];
     } else {
       return xr[j];
     }
   };
+  auto consumed = [&](int j) {  // slot j's buffer is free: request slot j + XD
+    if constexpr (XS && XD > 0) request(j + XD);
+  };
   char *yb = a.y[r];
 
   // ---- reduce-scatter: p-1 steps
   Acc msg[VEC];
   if (live(prev)) unpack<T>(xslot(0), msg);  // step 0 sends x_r[chunk r-1]
+  consumed(0);
 #pragma unroll
   for (int k = 0; k < PMAX - 1; ++k) {
     if (k + 1 >= p) break;
@@ -640,6 +656,7 @@ __global__ void __launch_bounds__(PMAX * L, MINB) rc_ring_link_kernel(const __gr
 #pragma unroll
       for (int e = 0; e < VEC; ++e) msg[e] = combine<OP>(msg[e], xv[e]);
     }
+    consumed(k + 1);
   }
   // the received chunk of the last step is r itself: finished
   uint4 fwd = make_uint4(0, 0, 0, 0);
@@ -670,7 +687,7 @@ __global__ void __launch_bounds__(PMAX * L, MINB) rc_ring_link_kernel(const __gr
   }
 }
 
-template <class T, int OP, int PMAX, int L, int MINB = 1, bool XS = false>
+template <class T, int OP, int PMAX, int L, int MINB = 1, bool XS = false, int XD = 0>
 cudaError_t launch_ring_link_t(const RingJob &job, uint64_t C, cudaStream_t s) {
   RingLinkParams a{};
   const int p = job.p;
@@ -687,8 +704,9 @@ cudaError_t launch_ring_link_t(const RingJob &job, uint64_t C, cudaStream_t s) {
   const uint64_t grid = (a.cv + L - 1) / L;
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffffull) return cudaErrorInvalidValue;
-  const size_t smem = ((size_t)2 * p * (VEC / 4) + (XS ? (size_t)p * p : 0)) * L * 16;
-  auto kern = rc_ring_link_kernel<T, OP, PMAX, L, MINB, XS>;
+  const size_t slots = XS ? (XD > 0 ? (size_t)XD : (size_t)p) : 0;  // staged slots per thread
+  const size_t smem = ((size_t)2 * p * (VEC / 4) + (size_t)p * slots) * L * 16;
+  auto kern = rc_ring_link_kernel<T, OP, PMAX, L, MINB, XS, XD>;
   if (smem > 48 * 1024) {  // opt in to the larger shared-memory carve-out, once per device
     static std::atomic<uint64_t> attr_set{0};
     int dev = 0;
@@ -696,7 +714,7 @@ cudaError_t launch_ring_link_t(const RingJob &job, uint64_t C, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_set.load() & bit)) {
-      const int most = (int)(((size_t)2 * PMAX * (VEC / 4) + (size_t)PMAX * PMAX) * L * 16);
+      const int most = (int)(((size_t)2 * PMAX * (VEC / 4) + (size_t)PMAX * (XD > 0 ? XD : PMAX)) * L * 16);
       err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
       if (err != cudaSuccess) return err;
       attr_set.fetch_or(bit);
@@ -707,8 +725,7 @@ cudaError_t launch_ring_link_t(const RingJob &job, uint64_t C, cudaStream_t s) {
 
 template <class T, int OP>
 cudaError_t launch_ring_link(const RingJob &job, uint64_t C, cudaStream_t s) {
-  // L = 32 lanes per rank: one warp per rank for p > 4; two warps per rank
-  // for p <= 4 keep the block at 256 threads.
+  // Lanes per rank: 16 for p > 4, 32 for p <= 4 (blocks of 128-256 threads).
   const int lanes = env_int("RC_RING_LANES", 0);
   const bool xs = env_int("RC_RING_XSMEM", 1) != 0;
   if (job.p <= 4) {
@@ -716,12 +733,21 @@ cudaError_t launch_ring_link(const RingJob &job, uint64_t C, cudaStream_t s) {
     if (lanes == 64) return launch_ring_link_t<T, OP, 4, 64>(job, C, s);
     return launch_ring_link_t<T, OP, 4, 32>(job, C, s);
   }
+  // staged-input window (RC_RING_XWIN): all p slots by default for p <= 8
+  // (a window of 4 or 6 measured no faster there); 4 slots for p > 8, where
+  // 16 slots per thread would hold the block to 2 per SM in bf16 (16 ranks x
+  // 8 MiB: 47.4 vs 52.1 us bf16, 46.2 vs 46.6 us fp32); 0 keeps every slot
+  const int win = env_int("RC_RING_XWIN", -1);
   if (job.p <= 8) {
+    if (xs && win == 4) return launch_ring_link_t<T, OP, 8, 16, 1, true, 4>(job, C, s);
+    if (xs && win == 6) return launch_ring_link_t<T, OP, 8, 16, 1, true, 6>(job, C, s);
     if (xs) return launch_ring_link_t<T, OP, 8, 16, 1, true>(job, C, s);
     if (lanes == 32) return launch_ring_link_t<T, OP, 8, 32>(job, C, s);
     return launch_ring_link_t<T, OP, 8, 16>(job, C, s);
   }
-  if (xs) return launch_ring_link_t<T, OP, 16, 16, 1, true>(job, C, s);
+  if (xs && win == 0) return launch_ring_link_t<T, OP, 16, 16, 1, true>(job, C, s);
+  if (xs && win == 8) return launch_ring_link_t<T, OP, 16, 16, 1, true, 8>(job, C, s);
+  if (xs) return launch_ring_link_t<T, OP, 16, 16, 1, true, 4>(job, C, s);
   return launch_ring_link_t<T, OP, 16, 16>(job, C, s);
 }
 
