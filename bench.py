@@ -72,7 +72,7 @@ WORKLOAD = ("ring/one-shot all_reduce workload: p=8 simulated ranks x 2,097,152 
 # previous call's dirty outputs are written back inside the captured launch
 # (bench.py --ncu-case OP --ncu-workload step).
 NCU_TRAFFIC = {
-    "ring_all_reduce": {"bytes": 67134208 + 63897600, "src": "209752cfdc9672f1"},
+    "ring_all_reduce": {"bytes": 67123200 + 63719168, "src": "f0a73279135321c7"},
     "all_reduce": {"bytes": 67107584 + 66091520, "src": "3194ac134632a10d"},
     "reduce_scatter": {"bytes": 67108864 + 5088256, "src": "3194ac134632a10d"},
     "all_gather": {"bytes": 4180224 + 28257536, "src": "02a6666765c86fcd"},
@@ -88,13 +88,13 @@ NCU_TRAFFIC = {
 # absolute times run about 10% long; the bench reports each collective's
 # share of this list times the live step time.
 NCU_IN_STEP = {
-    "all_reduce": {"us": 25.98, "dram": 67.1e6 + 65.7e6, "src": "3194ac134632a10d"},
-    "reduce_scatter": {"us": 16.77, "dram": 67.1e6 + 11.5e6, "src": "3194ac134632a10d"},
-    "all_gather": {"us": 9.69, "dram": 4.2e6 + 23.5e6, "src": "02a6666765c86fcd"},
-    "reduce": {"us": 17.62, "dram": 67.1e6 + 16.9e6, "src": "3194ac134632a10d"},
-    "broadcast": {"us": 12.68, "dram": 8.4e6 + 46.5e6, "src": "02a6666765c86fcd"},
-    "ring_all_reduce": {"us": 26.08, "dram": 65.1e6 + 70.2e6, "src": "209752cfdc9672f1"},
-    "hier_all_reduce": {"us": 25.37, "dram": 67.1e6 + 64.4e6, "src": "5eeac14585157d2b"},
+    "all_reduce": {"us": 25.46, "dram": 67.1e6 + 65.8e6, "src": "3194ac134632a10d"},
+    "reduce_scatter": {"us": 17.40, "dram": 67.1e6 + 13.8e6, "src": "3194ac134632a10d"},
+    "all_gather": {"us": 9.80, "dram": 4.2e6 + 23.3e6, "src": "02a6666765c86fcd"},
+    "reduce": {"us": 17.51, "dram": 67.1e6 + 14.1e6, "src": "3194ac134632a10d"},
+    "broadcast": {"us": 12.83, "dram": 8.4e6 + 46.9e6, "src": "02a6666765c86fcd"},
+    "ring_all_reduce": {"us": 26.09, "dram": 64.7e6 + 70.4e6, "src": "f0a73279135321c7"},
+    "hier_all_reduce": {"us": 25.47, "dram": 67.1e6 + 64.7e6, "src": "5eeac14585157d2b"},
 }
 
 
