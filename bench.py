@@ -660,10 +660,32 @@ def run_ours(args):
         eb.synchronize()
         e2e_s, e2e_bytes = reduce_over_ranks(ea.elapsed_time(eb) * 1e-3, step_bytes * e2e_k, world,
                                              device=dev)
+        # the PCIe ceiling of this pipeline: one step's host->device copies and
+        # one step's device->host copies running concurrently, as in the
+        # pipeline, without the collectives
+        torch.cuda.synchronize()
+        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pa.record(stream)
+        h2d_s.wait_event(pa)
+        d2h_s.wait_event(pa)
+        for _ in range(e2e_k):
+            with torch.cuda.stream(h2d_s):
+                for d, h in zip(bufs[0], host_in):
+                    d.copy_(h, non_blocking=True)
+            with torch.cuda.stream(d2h_s):
+                for h, d in zip(host_out, flat_outs):
+                    h.copy_(d, non_blocking=True)
+        stream.wait_stream(h2d_s)
+        stream.wait_stream(d2h_s)
+        pb.record(stream)
+        pb.synchronize()
+        copies_s = pa.elapsed_time(pb) * 1e-3 / e2e_k
         e2e = {"value": round(e2e_bytes / e2e_s / 1e9, 2), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "pipelined": "H2D of step k+1 on one stream overlaps D2H of step k on another "
-                            "(double-buffered device inputs)"}
+                            "(double-buffered device inputs)",
+               "copies_only_ms_per_step": round(copies_s * 1e3, 4),
+               "pcie_ceiling_gbs": round(step_bytes / copies_s / 1e9, 2)}
 
     if world > 1:
         import torch.distributed as dist
