@@ -713,6 +713,7 @@ def run_ours(args):
                       "in_sequence_us": round(seq_s[nm][1] * 1e6, 2),
                       "in_sequence_frac_of_measured_hbm": round(b / seq_s[nm][1] / 1e9 / peak, 4),
                       "repeated_frac_of_measured_hbm": round(b / rep_s[nm] / 1e9 / peak, 4),
+                      "repeated_frac_of_pages_8tbs": round(b / rep_s[nm] / 1e9 / PAGES_HBM_GBS, 4),
                       "isolated_us": round(ti * 1e6, 2),
                       "isolated_frac_of_measured_hbm": round(b / ti / 1e9 / peak, 4)}
     # in-step durations: each collective's share of the ncu launch list of the
